@@ -1,0 +1,136 @@
+"""fp64 CPU oracle for the Wan2.2 DiT self-attention path.
+
+TEST INFRASTRUCTURE ONLY: the tests, the package smoke check and the bench's
+CPU-baseline leg may import this; the product path never does. The arithmetic
+lives in ``wan_oracle.c`` (plain C, fp64, OpenMP over independent rows); this
+module builds it with gcc and marshals arrays through ctypes.
+
+bf16 tensors are exchanged as torch.bfloat16 tensors (their bit patterns are
+handed to C as uint16).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(HERE, "wan_oracle.c")
+LIB = os.path.join(HERE, "_build", "libwan_oracle.so")
+HEAD_DIM = 128
+SPLIT = (44, 42, 42)
+
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle (gcc, fp64, strict IEEE: no fast-math, no contraction)."""
+    os.makedirs(os.path.dirname(LIB), exist_ok=True)
+    if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < os.path.getmtime(SRC):
+        tmp = LIB + f".{os.getpid()}.tmp"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
+                               "-ffp-contract=off", "-fno-fast-math", SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, LIB)
+    return LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            P, I64, I32, D = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_double
+            lib.wan_oracle_round_bf16.argtypes = [D]
+            lib.wan_oracle_round_bf16.restype = D
+            lib.wan_oracle_f64_to_bf16.argtypes = [P, P, I64]
+            lib.wan_oracle_rmsnorm.argtypes = [P, I64, I64, I64, P, D, P]
+            lib.wan_oracle_rope.argtypes = [P, I64, I64, I32, I32, I32, D, P, I32]
+            lib.wan_oracle_qk_norm_rope.argtypes = [P, P, I64, I32, I32, I32, I32, P, P, D, D]
+            lib.wan_oracle_attention_rows.argtypes = [P, I64, I64, I32, D, P, I64, P]
+            _lib = lib
+    return _lib
+
+
+def _bits(t: torch.Tensor) -> np.ndarray:
+    assert t.dtype == torch.bfloat16
+    return np.ascontiguousarray(t.contiguous().view(torch.int16).numpy().view(np.uint16))
+
+
+def _ptr(a: np.ndarray) -> int:
+    return a.ctypes.data
+
+
+def round_bf16(x: float) -> float:
+    """fp64 -> nearest bf16 value, ties to even (as a Python float)."""
+    return _load().wan_oracle_round_bf16(float(x))
+
+
+def to_bf16(y) -> torch.Tensor:
+    """fp64 array -> bf16 tensor, each value rounded once, to nearest-even."""
+    y = np.ascontiguousarray(y, dtype=np.float64)
+    out = np.empty(y.shape, dtype=np.uint16)
+    _load().wan_oracle_f64_to_bf16(_ptr(y), _ptr(out), y.size)
+    return torch.from_numpy(out.view(np.int16)).view(torch.bfloat16)
+
+
+def rmsnorm(x: torch.Tensor, gamma: torch.Tensor, eps: float) -> np.ndarray:
+    """Step 1: x [n, d] bf16 -> x * rsqrt(mean(x^2) + eps) * gamma, fp64, unrounded."""
+    xb = _bits(x.reshape(-1, x.shape[-1]))
+    n, d = xb.shape
+    y = np.empty((n, d), dtype=np.float64)
+    g = _bits(gamma)
+    _load().wan_oracle_rmsnorm(_ptr(xb), n, d, d, _ptr(g), float(eps), _ptr(y))
+    return y
+
+
+def rope(y: np.ndarray, seq0: int, heads: int, grid, theta: float, split=SPLIT,
+         half_split: bool = False) -> np.ndarray:
+    """Step 3: rotate y [n, heads*128] fp64 for tokens seq0..seq0+n-1 of grid (F,H,W)."""
+    y = np.ascontiguousarray(y, dtype=np.float64).copy()
+    n = y.shape[0]
+    sp = (ctypes.c_int32 * 3)(*split)
+    _, H, W = grid
+    _load().wan_oracle_rope(_ptr(y), n, seq0, heads, H, W, float(theta),
+                            ctypes.cast(sp, ctypes.c_void_p), int(half_split))
+    return y
+
+
+def qk_norm_rope(qkv: torch.Tensor, grid, heads: int, gamma_q: torch.Tensor,
+                 gamma_k: torch.Tensor, eps: float, theta: float) -> torch.Tensor:
+    """Steps 1-3 on a packed [B, S, 3*heads*128] bf16 buffer; returns a new buffer."""
+    B, S, D3 = qkv.shape
+    F, H, W = grid
+    assert S == F * H * W and D3 == 3 * heads * HEAD_DIM
+    src = _bits(qkv)
+    dst = np.empty_like(src)
+    _load().wan_oracle_qk_norm_rope(_ptr(src), _ptr(dst), B, F, H, W, heads,
+                                    _ptr(_bits(gamma_q)), _ptr(_bits(gamma_k)),
+                                    float(eps), float(theta))
+    return torch.from_numpy(dst.view(np.int16)).view(torch.bfloat16).reshape(B, S, D3)
+
+
+def attention_rows(qkv: torch.Tensor, heads: int, rows, scale: float) -> np.ndarray:
+    """Step 4 for listed (b, h, i) query rows of a packed buffer; fp64 [n, 128]."""
+    B, S, D3 = qkv.shape
+    assert D3 == 3 * heads * HEAD_DIM
+    r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 3))
+    assert (r[:, 0] < B).all() and (r[:, 1] < heads).all() and (r[:, 2] < S).all() and (r >= 0).all()
+    out = np.empty((r.shape[0], HEAD_DIM), dtype=np.float64)
+    src = _bits(qkv)
+    _load().wan_oracle_attention_rows(_ptr(src), B, S, heads, float(scale), _ptr(r), r.shape[0],
+                                      _ptr(out))
+    return out
+
+
+def attention_full(qkv: torch.Tensor, heads: int, scale: float) -> np.ndarray:
+    """Step 4 for every row: fp64 [B, S, heads, 128]."""
+    B, S, _ = qkv.shape
+    b, h, i = np.meshgrid(np.arange(B), np.arange(heads), np.arange(S), indexing="ij")
+    rows = np.stack([b.transpose(0, 2, 1).ravel(), h.transpose(0, 2, 1).ravel(),
+                     i.transpose(0, 2, 1).ravel()], axis=1)
+    return attention_rows(qkv, heads, rows, scale).reshape(B, S, heads, HEAD_DIM)

@@ -1,0 +1,202 @@
+/*
+ * Wan2.2 DiT self-attention oracle: plain, slow, fp64 CPU code.
+ *
+ * TEST INFRASTRUCTURE ONLY. Nothing in the product path links or calls this
+ * file; only the tests, the package's smoke check and the bench's CPU-baseline
+ * leg do. It shares no code, header or table with the CUDA kernels.
+ *
+ * What it computes, step by step, in the order the pages give:
+ *
+ *  1. Q/K RMSNorm over the full hidden width D = heads*128 of each token
+ *     (review comments on TensorRT-LLM PR "[visual_gen] Optimize Wan2.2
+ *     Dataflow": the norm spans num_heads*head_dim, and the weight of channel
+ *     (head, dim) is gamma[head*head_dim + dim]).
+ *        r = 1 / sqrt(mean_c x_c^2 + eps),  y_c = x_c * r * gamma_c      (fp64)
+ *  2. Round y to bf16, round-to-nearest-even (same PR, "Fused Q/K Norm and
+ *     RoPE": the BF16 rounding point sits between the norm and RoPE).
+ *  3. 3D RoPE on adjacent pairs (2i, 2i+1) of each head: pairs [0,22) rotate
+ *     by the frame index, [22,43) by the row index, [43,64) by the column
+ *     index; within an axis of width d_a the j-th pair has frequency
+ *     theta^(-2j/d_a). Angle = position * frequency; rotation
+ *        (u, v) -> (u cos a - v sin a, u sin a + v cos a)          (fp64)
+ *     then round to bf16. V is copied unchanged. Token s sits at frame
+ *     s / (H*W), row (s / W) % H, column s % W.
+ *  4. Full bidirectional softmax attention per (batch, head):
+ *        o_i = sum_j softmax_j(scale * q_i . k_j) v_j                 (fp64)
+ *     evaluated as the plain definition (max-subtracted exponentials).
+ *
+ * The pair layout, axis order, frequency exponent, eps placement and rounding
+ * mode are readings of pages that leave them open; each is a parameter or a
+ * named constant here so that a test can flip it.
+ *
+ * bf16 values travel as their 16-bit patterns (uint16_t).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define HEAD_DIM 128
+
+static double bf16_to_f64(uint16_t b) {
+  uint32_t u = ((uint32_t)b) << 16;
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return (double)f;
+}
+
+/* Round a double to the nearest bf16 value (8 significant bits), ties to even.
+ * Written from the definition of the format: frexp gives x = m * 2^e with
+ * 0.5 <= |m| < 1, so m * 2^8 has exactly the 8 kept bits above the point. */
+double wan_oracle_round_bf16(double x) {
+  if (x == 0.0 || !isfinite(x)) return x;
+  int e;
+  double m = frexp(x, &e);
+  double r = nearbyint(ldexp(m, 8)); /* default rounding mode: nearest-even */
+  return ldexp(r, e - 8);
+}
+
+static uint16_t f64_to_bf16_bits(double x) {
+  /* x is already a bf16 value: the float conversion is exact. */
+  float f = (float)wan_oracle_round_bf16(x);
+  uint32_t u;
+  memcpy(&u, &f, sizeof u);
+  return (uint16_t)(u >> 16);
+}
+
+void wan_oracle_bf16_to_f64(const uint16_t* in, double* out, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) out[i] = bf16_to_f64(in[i]);
+}
+
+void wan_oracle_f64_to_bf16(const double* in, uint16_t* out, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) out[i] = f64_to_bf16_bits(in[i]);
+}
+
+/* Step 1 alone: y = x * r * gamma (fp64, not rounded) for n rows of width d.
+ * x: bf16 rows with a row stride of x_stride elements. */
+void wan_oracle_rmsnorm(const uint16_t* x, int64_t n, int64_t d, int64_t x_stride,
+                        const uint16_t* gamma, double eps, double* y) {
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < n; ++t) {
+    const uint16_t* row = x + t * x_stride;
+    double ss = 0.0;
+    for (int64_t c = 0; c < d; ++c) {
+      double v = bf16_to_f64(row[c]);
+      ss += v * v;
+    }
+    double r = 1.0 / sqrt(ss / (double)d + eps);
+    for (int64_t c = 0; c < d; ++c) y[t * d + c] = bf16_to_f64(row[c]) * r * bf16_to_f64(gamma[c]);
+  }
+}
+
+/* Which axis (0 frame, 1 row, 2 column) and which index within it a pair of
+ * a 128-wide head belongs to, for the split (d0, d1, d2) of head dims. */
+static void pair_axis(int pair, const int32_t split[3], int* axis, int* j) {
+  int p0 = split[0] / 2, p1 = split[1] / 2;
+  if (pair < p0) { *axis = 0; *j = pair; }
+  else if (pair < p0 + p1) { *axis = 1; *j = pair - p0; }
+  else { *axis = 2; *j = pair - p0 - p1; }
+}
+
+/* Rotate the pairs of one token's heads (heads x 128 doubles) for sequence
+ * index s of an F x H x W grid. half_split=0: adjacent pairs (2i, 2i+1), the
+ * reading taken; 1: pairs (i, i+64), kept only so a test can show the choice
+ * is observable. */
+static void rope_token(double* y, int64_t s, int32_t heads, int32_t H, int32_t W, double theta,
+                       const int32_t split[3], int32_t half_split) {
+  int64_t pos[3] = {s / ((int64_t)H * W), (s / W) % H, s % W};
+  for (int32_t h = 0; h < heads; ++h) {
+    double* head = y + (int64_t)h * HEAD_DIM;
+    for (int pair = 0; pair < HEAD_DIM / 2; ++pair) {
+      int axis, j;
+      pair_axis(pair, split, &axis, &j);
+      double freq = pow(theta, -2.0 * (double)j / (double)split[axis]);
+      double a = (double)pos[axis] * freq;
+      double c = cos(a), sn = sin(a);
+      int i0 = half_split ? pair : 2 * pair;
+      int i1 = half_split ? pair + HEAD_DIM / 2 : 2 * pair + 1;
+      double u = head[i0], v = head[i1];
+      head[i0] = u * c - v * sn;
+      head[i1] = u * sn + v * c;
+    }
+  }
+}
+
+/* Step 3 alone: rotate y (n tokens x heads x 128, fp64) in place, token t at
+ * sequence index seq0 + t; not rounded. */
+void wan_oracle_rope(double* y, int64_t n, int64_t seq0, int32_t heads, int32_t H, int32_t W,
+                     double theta, const int32_t split[3], int32_t half_split) {
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < n; ++t)
+    rope_token(y + t * heads * HEAD_DIM, seq0 + t, heads, H, W, theta, split, half_split);
+}
+
+/* Steps 1-3 for the packed buffer [B, S, 3, heads, 128] (bf16 bits):
+ * qkv_out gets normalised+rotated Q and K and a copy of V. */
+void wan_oracle_qk_norm_rope(const uint16_t* qkv_in, uint16_t* qkv_out, int64_t batch,
+                             int32_t F, int32_t H, int32_t W, int32_t heads,
+                             const uint16_t* gamma_q, const uint16_t* gamma_k, double eps,
+                             double theta) {
+  const int32_t split[3] = {44, 42, 42};
+  const int64_t S = (int64_t)F * H * W, D = (int64_t)heads * HEAD_DIM, D3 = 3 * D;
+  memcpy(qkv_out, qkv_in, (size_t)(batch * S * D3) * sizeof(uint16_t));
+#pragma omp parallel
+  {
+    double* y = (double*)malloc((size_t)D * sizeof(double));
+#pragma omp for schedule(static)
+    for (int64_t bt = 0; bt < batch * S; ++bt) {
+      for (int which = 0; which < 2; ++which) { /* 0: Q, 1: K */
+        const uint16_t* x = qkv_in + bt * D3 + which * D;
+        const uint16_t* g = which == 0 ? gamma_q : gamma_k;
+        wan_oracle_rmsnorm(x, 1, D, D, g, eps, y);                           /* step 1 */
+        for (int64_t c = 0; c < D; ++c) y[c] = wan_oracle_round_bf16(y[c]);  /* step 2 */
+        rope_token(y, bt % S, heads, H, W, theta, split, 0);                 /* step 3 */
+        uint16_t* o = qkv_out + bt * D3 + which * D;
+        for (int64_t c = 0; c < D; ++c) o[c] = f64_to_bf16_bits(y[c]);
+      }
+    }
+    free(y);
+  }
+}
+
+/* Step 4 on listed query rows. qkv: packed bf16 [B, S, 3, heads, 128] holding
+ * the (already normalised and rotated) Q and K and V. rows: n triplets
+ * (b, h, i). out: n x 128 fp64, unrounded. */
+void wan_oracle_attention_rows(const uint16_t* qkv, int64_t batch, int64_t S, int32_t heads,
+                               double scale, const int64_t* rows, int64_t n, double* out) {
+  (void)batch;
+  const int64_t D = (int64_t)heads * HEAD_DIM, D3 = 3 * D;
+#pragma omp parallel
+  {
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t r = 0; r < n; ++r) {
+      int64_t b = rows[3 * r], h = rows[3 * r + 1], i = rows[3 * r + 2];
+      const uint16_t* base = qkv + b * S * D3;
+      double q[HEAD_DIM];
+      for (int d = 0; d < HEAD_DIM; ++d) q[d] = bf16_to_f64(base[i * D3 + h * HEAD_DIM + d]);
+      /* pass 1: the largest logit */
+      double m = -INFINITY;
+      for (int64_t j = 0; j < S; ++j) {
+        const uint16_t* k = base + j * D3 + D + h * HEAD_DIM;
+        double dot = 0.0;
+        for (int d = 0; d < HEAD_DIM; ++d) dot += q[d] * bf16_to_f64(k[d]);
+        double l = dot * scale;
+        if (l > m) m = l;
+      }
+      /* pass 2: exponentials, their sum and the weighted sum of V */
+      double acc[HEAD_DIM];
+      for (int d = 0; d < HEAD_DIM; ++d) acc[d] = 0.0;
+      double sum = 0.0;
+      for (int64_t j = 0; j < S; ++j) {
+        const uint16_t* k = base + j * D3 + D + h * HEAD_DIM;
+        const uint16_t* v = base + j * D3 + 2 * D + h * HEAD_DIM;
+        double dot = 0.0;
+        for (int d = 0; d < HEAD_DIM; ++d) dot += q[d] * bf16_to_f64(k[d]);
+        double w = exp(dot * scale - m);
+        sum += w;
+        for (int d = 0; d < HEAD_DIM; ++d) acc[d] += w * bf16_to_f64(v[d]);
+      }
+      for (int d = 0; d < HEAD_DIM; ++d) out[r * HEAD_DIM + d] = acc[d] / sum;
+    }
+  }
+}

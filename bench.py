@@ -1,0 +1,376 @@
+#!/usr/bin/env python
+"""Benchmark: Wan2.2 DiT self-attention hot path on B200.
+
+One step = the whole path on one batch of the workload: Q/K RMSNorm + bf16
+round + 3D RoPE in place on the packed [Q|K|V] buffer, then softmax attention
+(``wan_dit_attn``: two kernels chained on one stream). Default workload: the
+Wan2.2-A14B 832x480, 81-frame clip with its CFG batch of 2 (grid 21x30x52 =
+32760 tokens, 40 heads x 128), synthetic seeded data.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0). ``value`` is attention TFLOP/s over whole steps
+(4*B*heads*S^2*128 FLOP per step / device time per step, all ranks); the
+line also carries per-kernel figures (attention TFLOP/s, norm+RoPE GB/s),
+the roofline of the dominant kernel, an end-to-end figure through host
+buffers, clocks seen during the timed region, and the oracle's CPU time.
+With N > 1 every rank runs an independent replica (the path does not shard):
+scaling is weak and ``value`` sums all ranks' work over the slowest rank's time.
+
+``--impl reference`` times the fp64 CPU oracle (the reference arm) on a
+bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import wan_inputs as wi  # noqa: E402
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+ATTN_SRC = os.path.join(ROOT, "video_diffusion_transformer_packed_b200", "csrc", "attn_fwd.cu")
+NORM_SRC = os.path.join(ROOT, "video_diffusion_transformer_packed_b200", "csrc", "qk_norm_rope.cu")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=wi.BENCH_WORKLOAD.name, choices=sorted(wi.BY_NAME))
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def sha256(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
+
+
+def profiled_traffic(kernel: str, src: str):
+    """DRAM bytes per launch from the committed ncu summary of `kernel`, if the
+    summary was taken on the current kernel source; else None."""
+    for fn in sorted(os.listdir(os.path.join(ROOT, "profiles"))) if os.path.isdir(os.path.join(ROOT, "profiles")) else []:
+        if not fn.startswith(kernel):
+            continue
+        txt = open(os.path.join(ROOT, "profiles", fn)).read()
+        m_sha = re.search(r"kernel_source_sha256\s*[:=]\s*([0-9a-f]{64})", txt)
+        m_tr = re.search(r"traffic_per_launch_bytes\s*[:=]\s*([0-9.eE+]+)", txt)
+        if m_sha and m_tr and m_sha.group(1) == sha256(src):
+            return float(m_tr.group(1))
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.proc = None
+        self.device = device
+
+    def start(self):
+        try:
+            props = torch.cuda.get_device_properties(self.device)
+            ident = "GPU-" + str(props.uuid) if getattr(props, "uuid", None) else str(self.device)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", ident], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+                power.append(float(f[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        busy = [s for s, p in zip(sm, power) if p > 0.5 * max(power)] or sm
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": max(power)}
+
+
+# ------------------------------------------------------------------ CPU oracle
+def oracle_sample(w, qkv, gq, gk, target_s: float):
+    """Times the oracle on a bounded sample of the workload: attention for n
+    query rows spread over (batch, head) pairs plus norm+RoPE for the matching
+    share of tokens (n / heads). Returns (TFLOP/s, seconds, description)."""
+    import numpy as np
+    import oracle
+    S, H = w.seq_len, w.heads
+    g = torch.Generator().manual_seed(1234)
+
+    def rows_for(n):
+        b = torch.randint(w.batch, (n,), generator=g)
+        h = torch.randint(H, (n,), generator=g)
+        i = torch.randint(S, (n,), generator=g)
+        return np.stack([b.numpy(), h.numpy(), i.numpy()], axis=1).astype(np.int64)
+
+    def run(n):
+        rows = rows_for(n)
+        ntok = max(1, n // H)
+        toks = np.stack([rows[:ntok, 0], rows[:ntok, 2]], axis=1)
+        t0 = time.perf_counter()
+        oracle.qk_norm_rope_tokens(qkv, w.grid, H, gq, gk, wi.EPS, wi.THETA, toks)
+        oracle.attention_rows(qkv, H, rows, 1.0 / 128 ** 0.5)
+        return time.perf_counter() - t0
+
+    oracle.build()
+    run(8)  # warm the library and threads
+    n0 = 16
+    t = run(n0)
+    n = int(max(n0, min(200000, n0 * target_s / max(t, 1e-6))))
+    t = run(n)
+    flop = n * 4.0 * S * wi.HEAD_DIM
+    desc = (f"{n} query rows of random (batch, head) pairs at S={S} plus norm+RoPE of {max(1, n // H)} "
+            f"tokens (the same share of the step), fp64 oracle")
+    return flop / t / 1e12, t, desc
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# -------------------------------------------------------------- reference arm
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = wi.BY_NAME[args.workload]
+    qkv, gq, gk = wi.inputs_for(w, seed=0)
+    per_step = max(1.0, 150.0 / max(1, args.steps + args.warmup))
+    vals, times, desc = [], [], ""
+    for k in range(args.warmup + args.steps):
+        v, t, desc = oracle_sample(w, qkv, gq, gk, per_step)
+        if k >= args.warmup:
+            vals.append(v)
+            times.append(t)
+    value = statistics.mean(vals)
+    cores = cpu_cores()
+    line = {
+        "impl": "reference", "metric": "self-attn TFLOP/s (% of B200 bf16 peak) at Wan 480p/81f; norm+RoPE GB/s",
+        "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * statistics.mean(times), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {**w.describe(), "sample": desc},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# -------------------------------------------------------------------- our arm
+def run_ours(args):
+    import video_diffusion_transformer_packed_b200 as wan
+    from video_diffusion_transformer_packed_b200 import build as wan_build
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (B200)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+        pg = dist
+    if rank == 0:
+        wan_build.build()
+    if pg is not None:
+        pg.barrier()
+    wan.load_library()
+
+    w = wi.BY_NAME[args.workload]
+    qkv_h, gq_h, gk_h = wi.inputs_for(w, seed=0)
+    qkv_pinned = torch.empty_like(qkv_h).pin_memory()
+    qkv_pinned.copy_(qkv_h)
+    qkv = qkv_pinned.to(dev)
+    gq, gk = gq_h.to(dev), gk_h.to(dev)
+    out = torch.empty((w.batch, w.seq_len, w.dim), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def step():
+        wan.dit_attn(qkv, w.grid, w.heads, gq, gk, out=out, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            step()
+    stream.synchronize()
+    if wan.device_error(stream) != 0:
+        raise SystemExit("attention kernel reported a device timeout during warm-up")
+
+    # ---- timed region: K whole steps, barrier + sync on both sides, device events
+    sampler = ClockSampler(local)
+    sampler.start()
+    if pg is not None:
+        pg.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    e1.synchronize()
+    torch.cuda.synchronize()
+    if pg is not None:
+        pg.barrier()
+    clocks = sampler.stop()
+    ms = e0.elapsed_time(e1)
+    if pg is not None:
+        t = torch.tensor([ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms = float(t.item())
+    if wan.device_error(stream) != 0:
+        raise SystemExit("attention kernel reported a device timeout during the timed region")
+    ms_step = ms / args.steps
+    value = world * w.attn_flop * args.steps / (ms / 1e3) / 1e12
+
+    # ---- per-kernel durations on the launching stream (separate calls, same work)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3 * args.steps)]
+    for k in range(args.steps):
+        ev[3 * k].record(stream)
+        wan.qk_norm_rope(qkv, w.grid, w.heads, gq, gk, stream=stream)
+        ev[3 * k + 1].record(stream)
+        wan.self_attention(qkv, w.heads, out=out, stream=stream)
+        ev[3 * k + 2].record(stream)
+    stream.synchronize()
+    t_norm = statistics.mean(ev[3 * k].elapsed_time(ev[3 * k + 1]) for k in range(args.steps))
+    t_attn = statistics.mean(ev[3 * k + 1].elapsed_time(ev[3 * k + 2]) for k in range(args.steps))
+    attn_tflops = w.attn_flop / (t_attn / 1e3) / 1e12
+    norm_gbs = w.norm_rope_bytes / (t_norm / 1e3) / 1e9
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        out_pinned = torch.empty((w.batch, w.seq_len, w.dim), dtype=torch.bfloat16).pin_memory()
+        h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            for k in range(args.warmup + args.steps):
+                if k == args.warmup:
+                    stream.synchronize()
+                    h0.record(stream)
+                qkv.copy_(qkv_pinned, non_blocking=True)
+                step()
+                out_pinned.copy_(out, non_blocking=True)
+            h1.record(stream)
+        stream.synchronize()
+        e2e_ms = h0.elapsed_time(h1)
+        if pg is not None:
+            t = torch.tensor([e2e_ms], device=dev)
+            pg.all_reduce(t, op=pg.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": world * w.attn_flop * args.steps / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": qkv.numel() * 2, "d2h_bytes_per_step": out.numel() * 2,
+               "ms_per_step": e2e_ms / args.steps}
+
+    peaks, peak_src = load_peaks()
+    tensor_peak = peaks["bf16_tflops_sustained"]
+    roofline = {
+        "kernel": "attn_fwd", "bound": "tensor", "achieved": attn_tflops, "peak": tensor_peak,
+        "unit": "TFLOP/s", "frac": attn_tflops / tensor_peak,
+        "traffic": profiled_traffic("attn_fwd", ATTN_SRC),
+        "peak_source": f"{peak_src} bf16 sustained (kernel timed inside seconds-long loops)",
+        "frac_of_burst_peak": attn_tflops / peaks["bf16_tflops"],
+        "algorithmic_flop_per_launch": w.attn_flop, "avg_launch_ms": t_attn,
+    }
+    norm_roofline = {
+        "kernel": "qk_norm_rope", "bound": "hbm", "achieved": norm_gbs, "peak": peaks["hbm_gbs"],
+        "unit": "GB/s", "frac": norm_gbs / peaks["hbm_gbs"],
+        "traffic": profiled_traffic("qk_norm_rope", NORM_SRC),
+        "algorithmic_bytes_per_launch": w.norm_rope_bytes, "avg_launch_ms": t_norm,
+        "peak_source": f"{peak_src} copy bandwidth",
+    }
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, t, desc = oracle_sample(w, qkv_h, gq_h, gk_h, args.cpu_seconds)
+        cpu = {"value": v, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle", "sample": desc,
+               "seconds": t}
+
+    if pg is not None:
+        pg.barrier()
+        pg.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": "self-attn TFLOP/s (% of B200 bf16 peak) at Wan 480p/81f; norm+RoPE GB/s",
+        "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {**w.describe(), "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": f"inputs larger than L2 ({qkv.numel() * 2 / 1e9:.2f} GB packed QKV per step)",
+                   "step": "wan_dit_attn: qk_norm_rope in place, then attention (PDL-chained)"},
+        "attn_tflops": attn_tflops, "attn_frac_of_peak": attn_tflops / tensor_peak,
+        "norm_rope_gbs": norm_gbs, "norm_rope_frac_of_hbm": norm_gbs / peaks["hbm_gbs"],
+        "roofline": roofline, "roofline_norm_rope": norm_roofline,
+        "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
+        "gpu_launches": 2 * args.steps,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,142 @@
+/*
+ * wan_attn.h -- C ABI of the Wan2.2 DiT self-attention hot path on B200 (sm_100a).
+ *
+ * The path (one DiT block's self-attention over video tokens, after the fused
+ * QKV projection):
+ *
+ *   packed [Q|K|V] --(1) Q/K RMSNorm over the full hidden width, bf16 round,
+ *                        3D RoPE, in place--> --(2) softmax attention--> out
+ *
+ * Sources for what is computed:
+ *  - Packed storage, strided Q/K reads, in-place update that keeps the shared
+ *    [Q | K | V] allocation, and the bf16 rounding point between the norm and
+ *    RoPE: TensorRT-LLM PR "[visual_gen] Optimize Wan2.2 Dataflow", section 1
+ *    "Preserve Packed QKV Storage Through Q/K Normalization and RoPE" and
+ *    "Fused Q/K Norm and RoPE" (FP32 accumulation -> BF16 -> FP32 RoPE -> BF16).
+ *  - Norm over num_heads*head_dim (5120 for A14B), weight index
+ *    head*head_dim + dim: the review comments on that PR.
+ *  - Token sequence S = F*H*W of the DiT grid and the bidirectional,
+ *    all-pairs attention whose cost grows as S^2: AWS Neuron "Optimizing
+ *    High-Quality Offline Video Generation", "Grounding in an output spec" and
+ *    "Context parallelism".
+ *  - 40 heads x 128 at S = 75600: the PR's "Packed QKV Profiling Details".
+ *  - head_dim 128 as a requirement of the Blackwell attention path: vLLM-Omni
+ *    "Wan2.2 Text-to-Video" recipe, Skip-Softmax requirements.
+ *  - Error instead of silent fallback: the same recipe ("raises rather than
+ *    silently degrading").
+ *
+ * Layouts (all row-major, bf16 = IEEE bfloat16 bit patterns):
+ *  - qkv:   [batch][S][3][heads][128]. Q of (b, s, h) starts at element
+ *           ((b*S + s)*3*D + h*128), K at +D, V at +2D, with D = heads*128.
+ *  - out:   [batch][S][heads][128], i.e. [batch][S][D].
+ *  - gamma: [D] (Q and K each), channel c = head*128 + dim.
+ *  - Token s of an F x H x W grid sits at frame s/(H*W), row (s/W)%H,
+ *    column s%W (width fastest).
+ *
+ * RoPE reading: head dims [0,44) rotate with the frame index, [44,86) with the
+ * row, [86,128) with the column; pairs are adjacent elements (2i, 2i+1); the
+ * j-th pair of an axis of width d_a has angle pos * theta^(-2j/d_a).
+ *
+ * Ownership and execution: the caller owns every buffer; the library
+ * allocates no device memory. Calls are asynchronous on `stream` (a
+ * cudaStream_t; NULL is the legacy default stream) and do not synchronise.
+ * Arguments are validated before anything is launched; on any error status
+ * nothing has been launched and no buffer has been written.
+ *
+ * Device requirement: compute capability 10.0 (B200, sm_100a); anything else
+ * returns WAN_ERR_UNSUPPORTED_DEVICE. There is no fallback path.
+ */
+#ifndef WAN_ATTN_H_
+#define WAN_ATTN_H_
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define WAN_API __attribute__((visibility("default")))
+#else
+#define WAN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  WAN_OK = 0,
+  WAN_ERR_NULL = 1,               /* a required pointer is NULL */
+  WAN_ERR_ALIGN = 2,              /* a pointer is not 16-byte aligned */
+  WAN_ERR_SHAPE = 3,              /* batch/grid/heads out of range, or overflow */
+  WAN_ERR_HEAD_DIM = 4,           /* head_dim != 128 */
+  WAN_ERR_PARAM = 5,              /* eps/theta/scale not finite or out of range */
+  WAN_ERR_UNSUPPORTED_DEVICE = 6, /* current device is not compute capability 10.0 */
+  WAN_ERR_LAUNCH = 7,             /* the CUDA runtime rejected a launch */
+  WAN_ERR_DEVICE_TIMEOUT = 8,     /* a kernel's bounded wait gave up (see wan_device_error) */
+  WAN_ERR_ALIAS = 9               /* out overlaps qkv */
+} wan_status;
+
+/* Largest head count accepted (hidden width 64*128 = 8192). */
+#define WAN_MAX_HEADS 64
+#define WAN_HEAD_DIM 128
+
+/* Static, human-readable text for a status code. Never NULL. */
+WAN_API const char* wan_status_string(int32_t status);
+
+/* Version of this ABI (bumped on any signature change). */
+WAN_API int32_t wan_abi_version(void);
+
+/*
+ * (1) Q/K RMSNorm + bf16 round + 3D RoPE, IN PLACE on the packed buffer.
+ *   For every token and X in {Q, K}:
+ *     r = 1/sqrt(mean_{c<D} X_c^2 + eps)      (fp32 accumulation)
+ *     y_c = bf16_rne(X_c * r * gamma_X[c])
+ *     pairs of y rotated by the token's (frame,row,column) angles in fp32,
+ *     then rounded to bf16 and written back over X.
+ *   V is neither read nor written.
+ * qkv      device pointer, bf16 [batch][F*H*W][3*heads*128], 16-byte aligned.
+ * gamma_q, gamma_k  device pointers, bf16 [heads*128], 16-byte aligned.
+ * batch >= 1; F, H, W >= 1 with F*H*W < 2^31; 1 <= heads <= WAN_MAX_HEADS;
+ * head_dim == 128; eps > 0 finite; theta > 1 finite.
+ */
+WAN_API int32_t wan_qk_norm_rope(void* qkv, int64_t batch, int32_t F, int32_t H, int32_t W,
+                         int32_t heads, int32_t head_dim, const void* gamma_q,
+                         const void* gamma_k, float eps, float theta, void* stream);
+
+/*
+ * (2) Full bidirectional softmax attention per (batch, head), reading Q, K and
+ *   V straight from the packed buffer (no repack):
+ *     out[b, i, h, :] = sum_j softmax_j(scale * q_i . k_j) v_j
+ *   bf16 operands, fp32 accumulation, probabilities rounded to bf16 before
+ *   the PV product, output rounded to bf16.
+ * qkv      device pointer, bf16 [batch][seq_len][3*heads*128], 16-byte aligned.
+ * out      device pointer, bf16 [batch][seq_len][heads*128], 16-byte aligned,
+ *          must not overlap qkv.
+ * scale    > 0, or <= 0 to mean 1/sqrt(head_dim).
+ * batch >= 1, 1 <= seq_len < 2^31, 1 <= heads <= WAN_MAX_HEADS, head_dim == 128.
+ */
+WAN_API int32_t wan_self_attention(const void* qkv, void* out, int64_t batch, int64_t seq_len,
+                           int32_t heads, int32_t head_dim, float scale, void* stream);
+
+/*
+ * (1) then (2) on one stream, the second launch chained to the first with
+ * programmatic dependent launch so its prologue overlaps the first's tail.
+ * Same arguments and in-place semantics as the two calls above, with
+ * seq_len = F*H*W. All arguments are validated before either launch.
+ */
+WAN_API int32_t wan_dit_attn(void* qkv, void* out, int64_t batch, int32_t F, int32_t H, int32_t W,
+                     int32_t heads, int32_t head_dim, const void* gamma_q, const void* gamma_k,
+                     float eps, float theta, float scale, void* stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the device-side error word
+ * that the attention kernel sets when one of its bounded waits gives up.
+ * *code receives 0 when no wait gave up, otherwise a nonzero site code.
+ * Returns WAN_ERR_DEVICE_TIMEOUT when *code != 0, WAN_ERR_NULL when code is
+ * NULL, WAN_ERR_LAUNCH when the synchronisation reports a CUDA error.
+ */
+WAN_API int32_t wan_device_error(void* stream, int32_t* code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WAN_ATTN_H_ */

@@ -51,6 +51,8 @@ def _load():
             lib.wan_oracle_rmsnorm.argtypes = [P, I64, I64, I64, P, D, P]
             lib.wan_oracle_rope.argtypes = [P, I64, I64, I32, I32, I32, D, P, I32]
             lib.wan_oracle_qk_norm_rope.argtypes = [P, P, I64, I32, I32, I32, I32, P, P, D, D]
+            lib.wan_oracle_qk_norm_rope_tokens.argtypes = [P, I64, I32, I32, I32, I32, P, P, D, D,
+                                                           P, I64, P]
             lib.wan_oracle_attention_rows.argtypes = [P, I64, I64, I32, D, P, I64, P]
             _lib = lib
     return _lib
@@ -112,6 +114,22 @@ def qk_norm_rope(qkv: torch.Tensor, grid, heads: int, gamma_q: torch.Tensor,
                                     _ptr(_bits(gamma_q)), _ptr(_bits(gamma_k)),
                                     float(eps), float(theta))
     return torch.from_numpy(dst.view(np.int16)).view(torch.bfloat16).reshape(B, S, D3)
+
+
+def qk_norm_rope_tokens(qkv: torch.Tensor, grid, heads: int, gamma_q: torch.Tensor,
+                        gamma_k: torch.Tensor, eps: float, theta: float, tokens) -> torch.Tensor:
+    """Steps 1-3 for listed (b, s) tokens: bf16 [n, 2*heads*128] ([Q | K] per token)."""
+    B, S, D3 = qkv.shape
+    F, H, W = grid
+    assert S == F * H * W and D3 == 3 * heads * HEAD_DIM
+    tk = np.ascontiguousarray(np.asarray(tokens, dtype=np.int64).reshape(-1, 2))
+    assert (tk >= 0).all() and (tk[:, 0] < B).all() and (tk[:, 1] < S).all()
+    out = np.empty((tk.shape[0], 2 * heads * HEAD_DIM), dtype=np.uint16)
+    src = _bits(qkv)
+    _load().wan_oracle_qk_norm_rope_tokens(_ptr(src), B, F, H, W, heads, _ptr(_bits(gamma_q)),
+                                           _ptr(_bits(gamma_k)), float(eps), float(theta), _ptr(tk),
+                                           tk.shape[0], _ptr(out))
+    return torch.from_numpy(out.view(np.int16)).view(torch.bfloat16)
 
 
 def attention_rows(qkv: torch.Tensor, heads: int, rows, scale: float) -> np.ndarray:

@@ -131,13 +131,24 @@ void wan_oracle_rope(double* y, int64_t n, int64_t seq0, int32_t heads, int32_t 
     rope_token(y + t * heads * HEAD_DIM, seq0 + t, heads, H, W, theta, split, half_split);
 }
 
+/* Steps 1-3 for one token: x (bf16 Q or K row of width heads*128) at
+ * sequence index s -> o (bf16). y is a scratch row of heads*128 doubles. */
+static void norm_rope_row(const uint16_t* x, uint16_t* o, double* y, int64_t s, int32_t heads,
+                          int32_t H, int32_t W, const uint16_t* gamma, double eps, double theta) {
+  const int32_t split[3] = {44, 42, 42};
+  const int64_t D = (int64_t)heads * HEAD_DIM;
+  wan_oracle_rmsnorm(x, 1, D, D, gamma, eps, y);                           /* step 1 */
+  for (int64_t c = 0; c < D; ++c) y[c] = wan_oracle_round_bf16(y[c]);  /* step 2 */
+  rope_token(y, s, heads, H, W, theta, split, 0);                      /* step 3 */
+  for (int64_t c = 0; c < D; ++c) o[c] = f64_to_bf16_bits(y[c]);
+}
+
 /* Steps 1-3 for the packed buffer [B, S, 3, heads, 128] (bf16 bits):
  * qkv_out gets normalised+rotated Q and K and a copy of V. */
 void wan_oracle_qk_norm_rope(const uint16_t* qkv_in, uint16_t* qkv_out, int64_t batch,
                              int32_t F, int32_t H, int32_t W, int32_t heads,
                              const uint16_t* gamma_q, const uint16_t* gamma_k, double eps,
                              double theta) {
-  const int32_t split[3] = {44, 42, 42};
   const int64_t S = (int64_t)F * H * W, D = (int64_t)heads * HEAD_DIM, D3 = 3 * D;
   memcpy(qkv_out, qkv_in, (size_t)(batch * S * D3) * sizeof(uint16_t));
 #pragma omp parallel
@@ -145,15 +156,32 @@ void wan_oracle_qk_norm_rope(const uint16_t* qkv_in, uint16_t* qkv_out, int64_t 
     double* y = (double*)malloc((size_t)D * sizeof(double));
 #pragma omp for schedule(static)
     for (int64_t bt = 0; bt < batch * S; ++bt) {
-      for (int which = 0; which < 2; ++which) { /* 0: Q, 1: K */
-        const uint16_t* x = qkv_in + bt * D3 + which * D;
-        const uint16_t* g = which == 0 ? gamma_q : gamma_k;
-        wan_oracle_rmsnorm(x, 1, D, D, g, eps, y);                           /* step 1 */
-        for (int64_t c = 0; c < D; ++c) y[c] = wan_oracle_round_bf16(y[c]);  /* step 2 */
-        rope_token(y, bt % S, heads, H, W, theta, split, 0);                 /* step 3 */
-        uint16_t* o = qkv_out + bt * D3 + which * D;
-        for (int64_t c = 0; c < D; ++c) o[c] = f64_to_bf16_bits(y[c]);
-      }
+      norm_rope_row(qkv_in + bt * D3, qkv_out + bt * D3, y, bt % S, heads, H, W, gamma_q, eps, theta);
+      norm_rope_row(qkv_in + bt * D3 + D, qkv_out + bt * D3 + D, y, bt % S, heads, H, W, gamma_k,
+                    eps, theta);
+    }
+    free(y);
+  }
+}
+
+/* Steps 1-3 for listed tokens only: tokens holds n pairs (b, s); out gets n
+ * rows of [Q | K] (2 * heads * 128 bf16 each). */
+void wan_oracle_qk_norm_rope_tokens(const uint16_t* qkv_in, int64_t batch, int32_t F, int32_t H,
+                                    int32_t W, int32_t heads, const uint16_t* gamma_q,
+                                    const uint16_t* gamma_k, double eps, double theta,
+                                    const int64_t* tokens, int64_t n, uint16_t* out) {
+  (void)batch;
+  const int64_t S = (int64_t)F * H * W, D = (int64_t)heads * HEAD_DIM, D3 = 3 * D;
+#pragma omp parallel
+  {
+    double* y = (double*)malloc((size_t)D * sizeof(double));
+#pragma omp for schedule(static)
+    for (int64_t r = 0; r < n; ++r) {
+      const int64_t bt = tokens[2 * r] * S + tokens[2 * r + 1];
+      norm_rope_row(qkv_in + bt * D3, out + r * 2 * D, y, tokens[2 * r + 1], heads, H, W, gamma_q,
+                    eps, theta);
+      norm_rope_row(qkv_in + bt * D3 + D, out + r * 2 * D + D, y, tokens[2 * r + 1], heads, H, W,
+                    gamma_k, eps, theta);
     }
     free(y);
   }

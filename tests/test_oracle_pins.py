@@ -351,3 +351,14 @@ def test_full_chain_brute_force_tiny_grid():
             # one-ulp slack: the reference rotates in a different order of operations
             ulp = torch.ldexp(torch.ones_like(exp), torch.frexp(exp.abs().clamp_min(1e-30)).exponent - 8)
             assert bool(((got - exp).abs() <= ulp).all())
+
+
+def test_token_subset_equals_full_buffer():
+    w = wi.Workload("t", 2, (3, 4, 5), 2)
+    qkv, gq, gk = wi.inputs_for(w, seed=41)
+    full = oracle.qk_norm_rope(qkv, w.grid, 2, gq, gk, EPS, THETA)
+    toks = [(0, 0), (1, 59), (1, 17), (0, 33)]
+    sub = oracle.qk_norm_rope_tokens(qkv, w.grid, 2, gq, gk, EPS, THETA, toks)
+    D = 2 * HD
+    for r, (b, s) in enumerate(toks):
+        assert torch.equal(sub[r].view(torch.int16), full[b, s, :2 * D].view(torch.int16))

@@ -1,0 +1,169 @@
+"""Wan2.2 DiT self-attention hot path for B200 (sm_100a): Python binding.
+
+A thin ctypes layer over the C ABI in ``include/wan_attn.h`` (library
+``_lib/libwanattn.so``, built by ``python -m video_diffusion_transformer_packed_b200.build``).
+It only marshals arguments -- tensor pointers, sizes and the current CUDA
+stream -- and turns a nonzero status into ``WanError``. Every step of the
+path runs in the library's kernels; there is no other implementation here,
+and a missing library is an error, not a fallback.
+
+    qk_norm_rope(qkv, grid, heads, gamma_q, gamma_k)   # in place on qkv
+    out = self_attention(qkv, heads)
+    out = dit_attn(qkv, grid, heads, gamma_q, gamma_k)   # both, chained
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional, Sequence
+
+__all__ = ["WanError", "load_library", "library_path", "qk_norm_rope", "self_attention",
+           "dit_attn", "device_error", "HEAD_DIM", "EPS", "THETA", "STATUS"]
+
+HEAD_DIM = 128
+EPS = 1e-6
+THETA = 10000.0
+STATUS = {0: "WAN_OK", 1: "WAN_ERR_NULL", 2: "WAN_ERR_ALIGN", 3: "WAN_ERR_SHAPE",
+          4: "WAN_ERR_HEAD_DIM", 5: "WAN_ERR_PARAM", 6: "WAN_ERR_UNSUPPORTED_DEVICE",
+          7: "WAN_ERR_LAUNCH", 8: "WAN_ERR_DEVICE_TIMEOUT", 9: "WAN_ERR_ALIAS"}
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "_lib", "libwanattn.so")
+_lib = None
+_lock = threading.Lock()
+
+
+class WanError(RuntimeError):
+    """A nonzero wan_status from the library."""
+
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = load_library().wan_status_string(status).decode()
+        super().__init__(f"{where}: {STATUS.get(status, status)} ({msg})")
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library() -> ctypes.CDLL:
+    """Load libwanattn.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(_LIB_PATH):
+                raise RuntimeError(f"{_LIB_PATH} is missing: build it with "
+                                   "`python -m video_diffusion_transformer_packed_b200.build`")
+            lib = ctypes.CDLL(_LIB_PATH)
+            P, I64, I32, F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float
+            lib.wan_status_string.argtypes = [I32]
+            lib.wan_status_string.restype = ctypes.c_char_p
+            lib.wan_abi_version.argtypes = []
+            lib.wan_abi_version.restype = I32
+            lib.wan_qk_norm_rope.argtypes = [P, I64, I32, I32, I32, I32, I32, P, P, F, F, P]
+            lib.wan_qk_norm_rope.restype = I32
+            lib.wan_self_attention.argtypes = [P, P, I64, I64, I32, I32, F, P]
+            lib.wan_self_attention.restype = I32
+            lib.wan_dit_attn.argtypes = [P, P, I64, I32, I32, I32, I32, I32, P, P, F, F, F, P]
+            lib.wan_dit_attn.restype = I32
+            lib.wan_device_error.argtypes = [P, ctypes.POINTER(I32)]
+            lib.wan_device_error.restype = I32
+            _lib = lib
+    return _lib
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise WanError(status, where)
+
+
+def _stream(stream) -> int:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _check_packed(qkv, heads: int, grid=None) -> None:
+    """Shapes the C ABI cannot see (it takes raw pointers): refuse mismatches
+    here, before anything is launched."""
+    if qkv.dim() != 3 or qkv.shape[2] != 3 * heads * HEAD_DIM:
+        raise ValueError(f"qkv must be [B, S, 3*heads*{HEAD_DIM}], got {tuple(qkv.shape)}")
+    if grid is not None and grid[0] * grid[1] * grid[2] != qkv.shape[1]:
+        raise ValueError(f"grid {tuple(grid)} has {grid[0] * grid[1] * grid[2]} tokens, "
+                         f"qkv has {qkv.shape[1]}")
+
+
+def _check_out(out, qkv, heads: int) -> None:
+    if tuple(out.shape) != (qkv.shape[0], qkv.shape[1], heads * HEAD_DIM):
+        raise ValueError(f"out must be [B, S, heads*{HEAD_DIM}], got {tuple(out.shape)}")
+
+
+def _check_gamma(g, heads: int, name: str) -> None:
+    if g.numel() != heads * HEAD_DIM:
+        raise ValueError(f"{name} must have heads*{HEAD_DIM} elements, got {g.numel()}")
+
+
+def _bf16_cuda(t, name: str) -> int:
+    import torch
+    if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+        raise TypeError(f"{name} must be a contiguous bfloat16 CUDA tensor")
+    return t.data_ptr()
+
+
+def qk_norm_rope(qkv, grid: Sequence[int], heads: int, gamma_q, gamma_k, eps: float = EPS,
+                 theta: float = THETA, stream=None):
+    """Q/K RMSNorm + bf16 round + 3D RoPE in place on packed qkv [B, F*H*W, 3*heads*128]."""
+    F, H, W = grid
+    B = qkv.shape[0]
+    _check_packed(qkv, heads, grid)
+    _check_gamma(gamma_q, heads, "gamma_q")
+    _check_gamma(gamma_k, heads, "gamma_k")
+    _check(load_library().wan_qk_norm_rope(_bf16_cuda(qkv, "qkv"), B, F, H, W, heads, HEAD_DIM,
+                                           _bf16_cuda(gamma_q, "gamma_q"),
+                                           _bf16_cuda(gamma_k, "gamma_k"), eps, theta,
+                                           _stream(stream)), "wan_qk_norm_rope")
+    return qkv
+
+
+def self_attention(qkv, heads: int, out=None, scale: float = 0.0, stream=None):
+    """Softmax attention over packed qkv [B, S, 3*heads*128] -> out [B, S, heads*128]."""
+    import torch
+    _check_packed(qkv, heads)
+    B, S, _ = qkv.shape
+    if out is None:
+        out = torch.empty((B, S, heads * HEAD_DIM), dtype=torch.bfloat16, device=qkv.device)
+    _check_out(out, qkv, heads)
+    _check(load_library().wan_self_attention(_bf16_cuda(qkv, "qkv"), _bf16_cuda(out, "out"), B, S,
+                                             heads, HEAD_DIM, scale, _stream(stream)),
+           "wan_self_attention")
+    return out
+
+
+def dit_attn(qkv, grid: Sequence[int], heads: int, gamma_q, gamma_k, out=None, eps: float = EPS,
+             theta: float = THETA, scale: float = 0.0, stream=None):
+    """qk_norm_rope (in place on qkv) then self_attention, chained on one stream."""
+    import torch
+    F, H, W = grid
+    _check_packed(qkv, heads, grid)
+    _check_gamma(gamma_q, heads, "gamma_q")
+    _check_gamma(gamma_k, heads, "gamma_k")
+    B, S, _ = qkv.shape
+    if out is None:
+        out = torch.empty((B, S, heads * HEAD_DIM), dtype=torch.bfloat16, device=qkv.device)
+    _check_out(out, qkv, heads)
+    _check(load_library().wan_dit_attn(_bf16_cuda(qkv, "qkv"), _bf16_cuda(out, "out"), B, F, H, W,
+                                       heads, HEAD_DIM, _bf16_cuda(gamma_q, "gamma_q"),
+                                       _bf16_cuda(gamma_k, "gamma_k"), eps, theta, scale,
+                                       _stream(stream)), "wan_dit_attn")
+    return out
+
+
+def device_error(stream=None) -> int:
+    """Synchronise and return (and clear) the attention kernel's device error word."""
+    code = ctypes.c_int32(0)
+    st = load_library().wan_device_error(_stream(stream), ctypes.byref(code))
+    if st not in (0, 8):
+        raise WanError(st, "wan_device_error")
+    return code.value

@@ -1,0 +1,176 @@
+// abi.cu -- the extern "C" boundary (include/wan_attn.h): argument
+// validation, device check, and the launches. No allocation, no fallback.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/wan_attn.h"
+#include "wan_kernels.h"
+
+namespace {
+
+constexpr int32_t kAbiVersion = 1;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Compute capability 10.0 only: the kernels are built for sm_100a.
+int32_t check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return WAN_ERR_UNSUPPORTED_DEVICE;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+    return WAN_ERR_UNSUPPORTED_DEVICE;
+  }
+  return (major == 10 && minor == 0) ? WAN_OK : WAN_ERR_UNSUPPORTED_DEVICE;
+}
+
+int32_t check_heads(int32_t heads, int32_t head_dim) {
+  if (head_dim != WAN_HEAD_DIM) return WAN_ERR_HEAD_DIM;
+  if (heads < 1 || heads > WAN_MAX_HEADS) return WAN_ERR_SHAPE;
+  return WAN_OK;
+}
+
+int32_t check_tokens(int64_t batch, int64_t seq_len, int32_t heads) {
+  if (batch < 1 || seq_len < 1 || seq_len > INT32_MAX) return WAN_ERR_SHAPE;
+  // Elements of the packed buffer must fit comfortably in int64, and the
+  // attention grid (batch * heads * ceil(S/256)) in a 31-bit grid dimension.
+  const int64_t d3 = 3 * static_cast<int64_t>(heads) * WAN_HEAD_DIM;
+  if (batch > (INT64_MAX / 4) / (seq_len * d3)) return WAN_ERR_SHAPE;
+  if (batch > (int64_t)INT32_MAX) return WAN_ERR_SHAPE;
+  const int64_t ctas = batch * heads * ((seq_len + 255) / 256);
+  if (ctas > INT32_MAX) return WAN_ERR_SHAPE;
+  // TMA tensor-map limits: each dimension < 2^32 and strides < 2^40 bytes.
+  if (static_cast<uint64_t>(seq_len) * static_cast<uint64_t>(d3) * 2ull >= (1ull << 40))
+    return WAN_ERR_SHAPE;
+  return WAN_OK;
+}
+
+int32_t check_grid(int64_t batch, int32_t F, int32_t H, int32_t W, int32_t heads, int64_t* S) {
+  if (F < 1 || H < 1 || W < 1) return WAN_ERR_SHAPE;
+  const int64_t s = static_cast<int64_t>(F) * H * W;
+  if (s > INT32_MAX) return WAN_ERR_SHAPE;
+  *S = s;
+  return check_tokens(batch, s, heads);
+}
+
+int32_t check_norm_args(void* qkv, const void* gq, const void* gk, float eps, float theta) {
+  if (!qkv || !gq || !gk) return WAN_ERR_NULL;
+  if (!aligned16(qkv) || !aligned16(gq) || !aligned16(gk)) return WAN_ERR_ALIGN;
+  if (!(std::isfinite(eps) && eps > 0.f)) return WAN_ERR_PARAM;
+  if (!(std::isfinite(theta) && theta > 1.f)) return WAN_ERR_PARAM;
+  return WAN_OK;
+}
+
+int32_t check_attn_args(const void* qkv, const void* out, int64_t batch, int64_t S, int32_t heads,
+                        float scale) {
+  if (!qkv || !out) return WAN_ERR_NULL;
+  if (!aligned16(qkv) || !aligned16(out)) return WAN_ERR_ALIGN;
+  if (!std::isfinite(scale)) return WAN_ERR_PARAM;
+  const uint64_t d = static_cast<uint64_t>(heads) * WAN_HEAD_DIM;
+  const uint64_t qkv_bytes = static_cast<uint64_t>(batch) * S * 3 * d * 2;
+  const uint64_t out_bytes = static_cast<uint64_t>(batch) * S * d * 2;
+  const uint64_t a0 = reinterpret_cast<uintptr_t>(qkv), a1 = a0 + qkv_bytes;
+  const uint64_t b0 = reinterpret_cast<uintptr_t>(out), b1 = b0 + out_bytes;
+  if (a0 < b1 && b0 < a1) return WAN_ERR_ALIAS;
+  return WAN_OK;
+}
+
+#define WAN_TRY(expr)          \
+  do {                         \
+    const int32_t _s = (expr); \
+    if (_s != WAN_OK) return _s; \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+const char* wan_status_string(int32_t status) {
+  switch (status) {
+    case WAN_OK: return "ok";
+    case WAN_ERR_NULL: return "a required pointer is NULL";
+    case WAN_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+    case WAN_ERR_SHAPE: return "batch, token grid or head count out of range";
+    case WAN_ERR_HEAD_DIM: return "head_dim must be 128";
+    case WAN_ERR_PARAM: return "eps, theta or scale is not finite or out of range";
+    case WAN_ERR_UNSUPPORTED_DEVICE: return "the current device is not compute capability 10.0 (sm_100a)";
+    case WAN_ERR_LAUNCH: return "the CUDA runtime rejected a launch";
+    case WAN_ERR_DEVICE_TIMEOUT: return "a bounded wait inside the attention kernel gave up";
+    case WAN_ERR_ALIAS: return "out overlaps qkv";
+    default: return "unknown status";
+  }
+}
+
+int32_t wan_abi_version(void) { return kAbiVersion; }
+
+int32_t wan_qk_norm_rope(void* qkv, int64_t batch, int32_t F, int32_t H, int32_t W, int32_t heads,
+                         int32_t head_dim, const void* gamma_q, const void* gamma_k, float eps,
+                         float theta, void* stream) {
+  int64_t S = 0;
+  WAN_TRY(check_heads(heads, head_dim));
+  WAN_TRY(check_grid(batch, F, H, W, heads, &S));
+  WAN_TRY(check_norm_args(qkv, gamma_q, gamma_k, eps, theta));
+  WAN_TRY(check_device());
+  (void)cudaGetLastError();
+  if (wan::launch_qk_norm_rope(qkv, batch, F, H, W, heads, gamma_q, gamma_k, eps, theta,
+                               static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    return WAN_ERR_LAUNCH;
+  }
+  return WAN_OK;
+}
+
+int32_t wan_self_attention(const void* qkv, void* out, int64_t batch, int64_t seq_len,
+                           int32_t heads, int32_t head_dim, float scale, void* stream) {
+  WAN_TRY(check_heads(heads, head_dim));
+  WAN_TRY(check_tokens(batch, seq_len, heads));
+  WAN_TRY(check_attn_args(qkv, out, batch, seq_len, heads, scale));
+  WAN_TRY(check_device());
+  (void)cudaGetLastError();
+  wan::AttnPlan plan;
+  if (wan::plan_attn_fwd(qkv, out, batch, seq_len, heads, scale, &plan) != cudaSuccess) {
+    return WAN_ERR_LAUNCH;
+  }
+  if (wan::launch_attn_fwd(plan, static_cast<cudaStream_t>(stream), false) != cudaSuccess) {
+    return WAN_ERR_LAUNCH;
+  }
+  return WAN_OK;
+}
+
+int32_t wan_dit_attn(void* qkv, void* out, int64_t batch, int32_t F, int32_t H, int32_t W,
+                     int32_t heads, int32_t head_dim, const void* gamma_q, const void* gamma_k,
+                     float eps, float theta, float scale, void* stream) {
+  int64_t S = 0;
+  WAN_TRY(check_heads(heads, head_dim));
+  WAN_TRY(check_grid(batch, F, H, W, heads, &S));
+  WAN_TRY(check_norm_args(qkv, gamma_q, gamma_k, eps, theta));
+  WAN_TRY(check_attn_args(qkv, out, batch, S, heads, scale));
+  WAN_TRY(check_device());
+  (void)cudaGetLastError();
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  wan::AttnPlan plan;
+  if (wan::plan_attn_fwd(qkv, out, batch, S, heads, scale, &plan) != cudaSuccess) {
+    return WAN_ERR_LAUNCH;
+  }
+  if (wan::launch_qk_norm_rope(qkv, batch, F, H, W, heads, gamma_q, gamma_k, eps, theta, st) !=
+      cudaSuccess) {
+    return WAN_ERR_LAUNCH;
+  }
+  if (wan::launch_attn_fwd(plan, st, true) != cudaSuccess) {
+    return WAN_ERR_LAUNCH;
+  }
+  return WAN_OK;
+}
+
+int32_t wan_device_error(void* stream, int32_t* code) {
+  if (!code) return WAN_ERR_NULL;
+  *code = 0;
+  if (wan::read_and_clear_device_error(static_cast<cudaStream_t>(stream), code) != cudaSuccess) {
+    return WAN_ERR_LAUNCH;
+  }
+  return *code != 0 ? WAN_ERR_DEVICE_TIMEOUT : WAN_OK;
+}
+
+}  // extern "C"

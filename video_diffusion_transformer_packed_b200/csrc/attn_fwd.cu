@@ -1,0 +1,510 @@
+// attn_fwd.cu -- full bidirectional softmax attention over the packed Wan2.2
+// QKV buffer, head_dim 128, bf16 in / bf16 out, fp32 accumulation (sm_100a).
+//
+//   out[b, i, h, :] = sum_j softmax_j(scale * q_i . k_j) v_j
+//
+// The attention is the dominant cost of a DiT block: all-pairs over the
+// video tokens, S^2 work (AWS Neuron "Optimizing High-Quality Offline Video
+// Generation", "Context parallelism"); Q, K and V are read straight out of
+// the packed [Q | K | V] allocation with no repack (TensorRT-LLM PR
+// "[visual_gen] Optimize Wan2.2 Dataflow", "Packed QKV Profiling Details").
+//
+// Design (one CTA = one (batch, head) and two 128-row query tiles):
+//   warp 8      TMA producer: Q tiles once, then K_j / V_j tiles into a
+//               4-slot shared-memory ring (128-byte swizzle, 3D tensor map
+//               over [B][S][3D] so that rows past S read as zeros per batch).
+//   warp 9      MMA issuer (one thread): tcgen05.mma S_t = Q_t K_j^T into
+//               TMEM, then O_t += P_t V_j with P_t read from TMEM. The two
+//               query tiles ping-pong: while one tile's softmax runs, the
+//               tensor core works on the other tile.
+//   warps 0-3   softmax of tile 0, warps 4-7 softmax of tile 1: thread r owns
+//               query row r (TMEM lane r). Online softmax in base 2; the
+//               running max is only raised (and O rescaled in TMEM) when a
+//               tile's max exceeds it by more than 2^8, which keeps the
+//               result exact after the final division while skipping almost
+//               all rescales. P is rounded to bf16 and written over S in TMEM.
+// TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,384), O_1 [384,512).
+//
+// Every mbarrier wait is bounded (wall-clock limit); a wait that gives up
+// sets a block-wide abort flag and a device error word, and the block then
+// drains its own copies and MMAs, frees TMEM and exits.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "sm100.cuh"
+#include "wan_kernels.h"
+
+namespace wan {
+namespace {
+
+using namespace wan::sm100;
+
+constexpr int kBM = 128;  // query rows per tile
+constexpr int kBN = 128;  // keys per tile
+constexpr int kHD = 128;  // head dim
+constexpr int kStages = 4;
+constexpr int kTileBytes = kBM * kHD * 2;  // 32 KB: one 128 x 128 bf16 tile
+constexpr int kBoxBytes = kTileBytes / 2;  // 16 KB: 128 rows x 64 columns (one TMA box)
+constexpr int kThreads = 384;  // 3 warpgroups: softmax tile 0, softmax tile 1, load/MMA
+constexpr int kLoadWarp = 8;
+constexpr int kMmaWarp = 9;
+// Register split. The launch gives every thread kLaunchRegs (checked on the
+// host against the compiled kernel before any launch); the load/MMA
+// warpgroup gives registers back and the two softmax warpgroups take them:
+// 128*kCtlRegs + 256*kSoftmaxRegs must not exceed 384*kLaunchRegs.
+constexpr int kLaunchRegs = 168;
+constexpr int kCtlRegs = 72;
+constexpr int kSoftmaxRegs = 216;
+static_assert(128 * kCtlRegs + 256 * kSoftmaxRegs <= kThreads * kLaunchRegs, "register split");
+constexpr uint32_t kTmemCols = 512;
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
+constexpr float kRescaleThreshold = 8.0f;         // log2 of the largest tolerated growth
+
+// Shared memory map (offsets from a 1024-byte aligned base).
+constexpr int kOffQ = 0;                              // 2 tiles
+constexpr int kOffKV = kOffQ + 2 * kTileBytes;        // kStages tiles
+constexpr int kOffBar = kOffKV + kStages * kTileBytes;
+constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 2 + 1;  // q, kv full/empty, s, p, o, drain
+constexpr int kOffMisc = kOffBar + kNumBars * 8;
+constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + alignment slack
+
+// Error-word site codes.
+constexpr int kErrProducer = 1, kErrMma = 2, kErrSoftmax = 4, kErrEpilogue = 8, kErrDrain = 16;
+
+__device__ int g_attn_error_word;
+
+struct AttnParams {
+  uint16_t* out;
+  int32_t S;
+  int32_t heads;
+  int32_t D;
+  int32_t q_pairs;  // ceil(S / 256): CTAs per (batch, head)
+  int32_t n_kv;     // ceil(S / 128)
+  float scale_log2; // scale * log2(e)
+};
+
+// Barrier addresses (32-bit shared-memory addresses, 8 bytes apart).
+struct Bars {
+  uint32_t base;
+  __device__ __forceinline__ uint32_t q_full() const { return base; }
+  __device__ __forceinline__ uint32_t kv_full(int s) const { return base + 8 * (1 + s); }
+  __device__ __forceinline__ uint32_t kv_empty(int s) const { return base + 8 * (1 + kStages + s); }
+  __device__ __forceinline__ uint32_t s_full(int t) const { return base + 8 * (1 + 2 * kStages + t); }
+  __device__ __forceinline__ uint32_t p_full(int t) const { return base + 8 * (3 + 2 * kStages + t); }
+  __device__ __forceinline__ uint32_t o_full(int t) const { return base + 8 * (5 + 2 * kStages + t); }
+  __device__ __forceinline__ uint32_t drain() const { return base + 8 * (7 + 2 * kStages); }
+};
+static_assert(8 + 2 * kStages == kNumBars, "barrier count");
+
+__device__ __forceinline__ void flag_error(volatile int* abort, int site) {
+  *abort = 1;
+  atomicOr(&g_attn_error_word, site);
+}
+
+// ---------------------------------------------------------------- producer
+__device__ void run_producer(const CUtensorMap* tmap, const AttnParams& p, uint32_t smem,
+                             Bars bars, volatile int* abort, int* issued, int b, int h, int qp) {
+  grid_dependency_wait();  // the packed buffer may still be written by the norm kernel
+  const int xq = h * kHD, xk = p.D + h * kHD, xv = 2 * p.D + h * kHD;
+  mbar_arrive_expect_tx(bars.q_full(), 2 * kTileBytes);
+  for (int t = 0; t < 2; ++t) {
+    for (int half = 0; half < 2; ++half) {
+      tma_load_3d(smem + kOffQ + t * kTileBytes + half * kBoxBytes, tmap, bars.q_full(),
+                  xq + 64 * half, (2 * qp + t) * kBM, b);
+    }
+  }
+  bool ok = true;
+  const int items = 2 * p.n_kv;  // K_0, V_0, K_1, V_1, ...
+#pragma unroll 1
+  for (int i = 0; i < items; ++i) {
+    const int slot = i % kStages;
+    const int use = i / kStages;
+    if (use > 0 && !mbar_wait(bars.kv_empty(slot), (use - 1) & 1, abort, kWaitLimitNs)) {
+      ok = false;
+      break;
+    }
+    mbar_arrive_expect_tx(bars.kv_full(slot), kTileBytes);
+    const int x = (i & 1) ? xv : xk;
+    const int y = (i >> 1) * kBN;
+    const uint32_t dst = smem + kOffKV + slot * kTileBytes;
+    tma_load_3d(dst, tmap, bars.kv_full(slot), x, y, b);
+    tma_load_3d(dst + kBoxBytes, tmap, bars.kv_full(slot), x + 64, y, b);
+    issued[slot] = use + 1;
+  }
+  if (!ok) flag_error(abort, kErrProducer);
+}
+
+// After an abort, waits (bounded, ignoring the abort flag) for every copy the
+// producer started, so that no bulk copy lands after the block has exited.
+__device__ void drain_producer(Bars bars, const int* issued) {
+  for (int s = 0; s < kStages; ++s) {
+    if (issued[s] > 0 && !mbar_wait(bars.kv_full(s), (issued[s] - 1) & 1, nullptr, kWaitLimitNs)) {
+      atomicOr(&g_attn_error_word, kErrDrain);
+    }
+  }
+  if (!mbar_wait(bars.q_full(), 0, nullptr, kWaitLimitNs)) atomicOr(&g_attn_error_word, kErrDrain);
+}
+
+// -------------------------------------------------------------- MMA issuer
+__device__ void run_mma(const AttnParams& p, uint32_t smem, Bars bars, volatile int* abort,
+                        uint32_t tmem) {
+  constexpr uint32_t kIdescQK = idesc_bf16_f32(kBM, kBN, 0);
+  constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, kHD, 1);
+  // Descriptors are built once; a step only adds a byte offset (in 16-byte
+  // units) to the start-address field, which cannot carry out of its 14 bits
+  // because shared-memory addresses stay below 2^18.
+  //
+  // S_t = Q_t K^T: K = 128 head dims in 8 steps of 16; each 64-dim half of a
+  // tile is one 128-byte-swizzled box, and a 16-element step inside a box
+  // advances the start address by 32 bytes.
+  const uint64_t q_desc0 = smem_desc_sw128(smem + kOffQ, 16, 1024);
+  const uint64_t k_desc0 = smem_desc_sw128(smem + kOffKV, 16, 1024);
+  // V [key][dim] is an N-major B: 8-key groups 1024 bytes apart, the two
+  // 64-dim halves one box (16 KB) apart; a 16-key step advances 2048 bytes.
+  const uint64_t v_desc0 = smem_desc_sw128(smem + kOffKV, kBoxBytes, 1024);
+
+  auto issue_qk = [&](int t, int slot) {
+    const uint32_t a0 = (t * kTileBytes) >> 4;
+    const uint32_t b0 = (slot * kTileBytes) >> 4;
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      const uint32_t off = ((kk >> 2) * kBoxBytes + (kk & 3) * 32) >> 4;
+      mma_ss(tmem + t * 128, desc_add(q_desc0, a0 + off), desc_add(k_desc0, b0 + off), kIdescQK,
+             kk > 0 ? 1u : 0u);
+    }
+  };
+  // O_t += P_t V: P_t (bf16, 64 TMEM columns over S_t) is the A operand.
+  auto issue_pv = [&](int t, int slot, uint32_t acc) {
+    const uint32_t b0 = (slot * kTileBytes) >> 4;
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      mma_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, desc_add(v_desc0, b0 + kk * (2048 >> 4)),
+             kIdescPV, kk > 0 ? 1u : acc);
+    }
+  };
+  auto wait_item = [&](int i) -> bool {
+    return mbar_wait(bars.kv_full(i % kStages), (i / kStages) & 1, abort, kWaitLimitNs);
+  };
+
+  bool ok = mbar_wait(bars.q_full(), 0, abort, kWaitLimitNs) && wait_item(0);
+  if (ok) {
+    tc_fence_after();
+    issue_qk(0, 0);
+    mma_commit(bars.s_full(0));
+    issue_qk(1, 0);
+    mma_commit(bars.s_full(1));
+    mma_commit(bars.kv_empty(0));
+  }
+#pragma unroll 1
+  for (int j = 0; j < p.n_kv && ok; ++j) {
+    const int iv = 2 * j + 1, ik = 2 * j + 2;
+    const bool more = j + 1 < p.n_kv;
+    const uint32_t acc = j > 0 ? 1u : 0u;
+    if (!wait_item(iv) || !mbar_wait(bars.p_full(0), j & 1, abort, kWaitLimitNs)) { ok = false; break; }
+    tc_fence_after();
+    issue_pv(0, iv % kStages, acc);
+    if (more) {
+      if (!wait_item(ik)) { ok = false; break; }
+      tc_fence_after();
+      issue_qk(0, ik % kStages);
+      mma_commit(bars.s_full(0));
+    }
+    if (!mbar_wait(bars.p_full(1), j & 1, abort, kWaitLimitNs)) { ok = false; break; }
+    tc_fence_after();
+    issue_pv(1, iv % kStages, acc);
+    mma_commit(bars.kv_empty(iv % kStages));
+    if (more) {
+      issue_qk(1, ik % kStages);
+      mma_commit(bars.s_full(1));
+      mma_commit(bars.kv_empty(ik % kStages));
+    }
+  }
+  if (ok) {
+    mma_commit(bars.o_full(0));
+    mma_commit(bars.o_full(1));
+  } else {
+    flag_error(abort, kErrMma);
+  }
+  // Every MMA this thread issued completes before TMEM can be released.
+  mma_commit(bars.drain());
+  if (!mbar_wait(bars.drain(), 0, nullptr, kWaitLimitNs)) atomicOr(&g_attn_error_word, kErrDrain);
+}
+
+// ----------------------------------------------------------------- softmax
+__device__ void run_softmax(const AttnParams& p, Bars bars, volatile int* abort, uint32_t tmem,
+                            int t, int quarter, int lane, int b, int h, int qp) {
+  const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+  const uint32_t tS = tmem + lane_base + t * 128;
+  const uint32_t tO = tmem + lane_base + 256 + t * 128;
+  const float sl2 = p.scale_log2;
+  float m_run = -INFINITY;  // running max, already in scaled log2 units
+  float l_run = 0.f;
+  bool ok = true;
+
+#pragma unroll 1
+  for (int j = 0; j < p.n_kv; ++j) {
+    if (!mbar_wait(bars.s_full(t), j & 1, abort, kWaitLimitNs)) { ok = false; break; }
+    tc_fence_after();
+    uint32_t sr[128];  // raw fp32 scores of this thread's row
+    tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(sr + 0));
+    tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
+    tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(sr + 64));
+    tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(sr + 96));
+    tmem_wait_ld();
+    const int rem = p.S - j * kBN;  // valid keys in this tile
+    if (rem < kBN) {
+#pragma unroll
+      for (int c = 0; c < 128; ++c) sr[c] = c < rem ? sr[c] : __float_as_uint(-INFINITY);
+    }
+    float mx = __uint_as_float(sr[0]);
+#pragma unroll
+    for (int c = 1; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(sr[c]));
+    const float m_cand = mx * sl2;
+    const bool raise = m_cand > m_run + kRescaleThreshold;
+    float alpha = 1.f;
+    if (raise) {
+      alpha = ex2(m_run - m_cand);
+      m_run = m_cand;
+    }
+    l_run *= alpha;
+    if (j > 0 && __any_sync(0xffffffffu, raise)) {
+      // O_t is quiescent here: S_t's completion implies every earlier MMA
+      // (including the previous O_t += P V) has completed.
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tO + 32 * c, o);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+        tmem_st32(tO + 32 * c, o);
+      }
+      tmem_wait_st();
+    }
+    const float neg_m = -m_run;
+    float sum = 0.f;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      uint32_t pk[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const float p0 = ex2(fmaf(__uint_as_float(sr[64 * half + 2 * e]), sl2, neg_m));
+        const float p1 = ex2(fmaf(__uint_as_float(sr[64 * half + 2 * e + 1]), sl2, neg_m));
+        sum += p0 + p1;
+        pk[e] = pack_bf16x2(p0, p1);
+      }
+      tmem_st32(tS + 32 * half, pk);
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    mbar_arrive(bars.p_full(t));
+    l_run += sum;
+  }
+  if (!ok) {
+    flag_error(abort, kErrSoftmax);
+    return;
+  }
+  if (!mbar_wait(bars.o_full(t), 0, abort, kWaitLimitNs)) {
+    flag_error(abort, kErrEpilogue);
+    return;
+  }
+  tc_fence_after();
+  const float inv_l = 1.f / l_run;
+  const int row = (2 * qp + t) * kBM + quarter * 32 + lane;
+  uint16_t* dst = p.out + (static_cast<int64_t>(b) * p.S + row) * p.D + h * kHD;
+#pragma unroll 1
+  for (int c = 0; c < 4; ++c) {
+    uint32_t o[32];
+    tmem_ld32(tO + 32 * c, o);
+    tmem_wait_ld();
+    if (row < p.S) {
+      uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const float* f = reinterpret_cast<const float*>(o) + 8 * v;
+        d4[v] = make_uint4(pack_bf16x2(f[0] * inv_l, f[1] * inv_l), pack_bf16x2(f[2] * inv_l, f[3] * inv_l),
+                           pack_bf16x2(f[4] * inv_l, f[5] * inv_l), pack_bf16x2(f[6] * inv_l, f[7] * inv_l));
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t smem_base = smem_u32(smem);
+  const Bars bars{smem_base + kOffBar};
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kOffMisc);
+  volatile int* abort = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
+  int* issued = reinterpret_cast<int*>(smem + kOffMisc + 8);  // [kStages], producer-owned
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int qp = blockIdx.x % p.q_pairs;
+  const int bh = blockIdx.x / p.q_pairs;
+  const int b = bh / p.heads;
+  const int h = bh % p.heads;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bars.q_full(), 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bars.kv_full(s), 1);
+      mbar_init(bars.kv_empty(s), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bars.s_full(t), 1);
+      mbar_init(bars.p_full(t), 128);
+      mbar_init(bars.o_full(t), 1);
+    }
+    mbar_init(bars.drain(), 1);
+    *abort = 0;
+    for (int s = 0; s < kStages; ++s) issued[s] = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_holder, kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == kLoadWarp && lane == 0) tma_prefetch_desc(&tmap);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp >= 8) {
+    regs_decrease<kCtlRegs>();
+    if (warp == kLoadWarp) {
+      if (lane == 0) run_producer(&tmap, p, smem_base, bars, abort, issued, b, h, qp);
+    } else if (warp == kMmaWarp) {
+      if (lane == 0) run_mma(p, smem_base, bars, abort, tmem);
+    }
+    __syncwarp();
+  } else {
+    regs_increase<kSoftmaxRegs>();
+    run_softmax(p, bars, abort, tmem, warp >> 2, warp & 3, lane, b, h, qp);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kLoadWarp && lane == 0 && *abort) drain_producer(bars, issued);
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------- host
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess) {
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+  });
+  return fn;
+}
+
+}  // namespace
+
+cudaError_t plan_attn_fwd(const void* qkv, void* out, int64_t batch, int64_t seq_len,
+                          int32_t heads, float scale, AttnPlan* plan) {
+  static_assert(sizeof(CUtensorMap) == sizeof(plan->tmap), "tensor map size");
+  const int32_t S = static_cast<int32_t>(seq_len);
+  const int32_t D = heads * kHD;
+  auto encode = get_encode_fn();
+  if (!encode) return cudaErrorNotSupported;
+
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] {
+    // The register split inside the kernel is only safe when the compiled
+    // kernel launches with exactly kLaunchRegs registers per thread.
+    cudaFuncAttributes fa;
+    attr_err = cudaFuncGetAttributes(&fa, attn_fwd_kernel);
+    if (attr_err == cudaSuccess && fa.numRegs != kLaunchRegs) attr_err = cudaErrorInvalidKernelImage;
+    if (attr_err == cudaSuccess) {
+      attr_err = cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      kSmemBytes);
+    }
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+
+  // Packed buffer as a 3D tensor: x = channel (3D), y = token, z = batch.
+  // Boxes are 64 channels (128 bytes, the swizzle span) x 128 tokens.
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(3 * D), static_cast<cuuint64_t>(S),
+                        static_cast<cuuint64_t>(batch)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(3 * D) * 2,
+                           static_cast<cuuint64_t>(3 * D) * 2 * static_cast<cuuint64_t>(S)};
+  cuuint32_t box[3] = {64, kBM, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = encode(reinterpret_cast<CUtensorMap*>(plan->tmap), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                      const_cast<void*>(qkv), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+
+  plan->out = out;
+  plan->S = S;
+  plan->heads = heads;
+  plan->D = D;
+  plan->q_pairs = (S + 2 * kBM - 1) / (2 * kBM);
+  plan->n_kv = (S + kBN - 1) / kBN;
+  const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(kHD));
+  plan->scale_log2 = sc * 1.4426950408889634f;
+  plan->grid = batch * heads * static_cast<int64_t>(plan->q_pairs);
+  return cudaSuccess;
+}
+
+cudaError_t launch_attn_fwd(const AttnPlan& plan, cudaStream_t stream, bool pdl) {
+  AttnParams p;
+  p.out = static_cast<uint16_t*>(plan.out);
+  p.S = plan.S;
+  p.heads = plan.heads;
+  p.D = plan.D;
+  p.q_pairs = plan.q_pairs;
+  p.n_kv = plan.n_kv;
+  p.scale_log2 = plan.scale_log2;
+  CUtensorMap tmap;
+  memcpy(&tmap, plan.tmap, sizeof(tmap));
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(plan.grid));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, attn_fwd_kernel, tmap, p);
+}
+
+cudaError_t read_and_clear_device_error(cudaStream_t stream, int32_t* code) {
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return e;
+  int v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_attn_error_word, sizeof(int));
+  if (e != cudaSuccess) return e;
+  if (v != 0) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(g_attn_error_word, &zero, sizeof(int));
+    if (e != cudaSuccess) return e;
+  }
+  *code = v;
+  return cudaSuccess;
+}
+
+}  // namespace wan

@@ -1,0 +1,38 @@
+// wan_kernels.h -- host-side launchers of the two sm_100a kernels (internal to
+// the library; the public surface is include/wan_attn.h).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace wan {
+
+// Q/K RMSNorm + bf16 round + 3D RoPE, in place on the packed buffer.
+// Arguments are assumed validated by the ABI layer.
+cudaError_t launch_qk_norm_rope(void* qkv, int64_t batch, int32_t F, int32_t H, int32_t W,
+                                int32_t heads, const void* gamma_q, const void* gamma_k, float eps,
+                                float theta, cudaStream_t stream);
+
+// Everything the attention launch needs, prepared before anything is
+// launched (tensor-map encoding can fail; a launch after a successful plan
+// only fails if the runtime rejects it).
+struct AttnPlan {
+  alignas(64) unsigned char tmap[128];  // CUtensorMap over the packed buffer
+  void* out;
+  int32_t S, heads, D, q_pairs, n_kv;
+  float scale_log2;
+  int64_t grid;
+};
+
+cudaError_t plan_attn_fwd(const void* qkv, void* out, int64_t batch, int64_t seq_len,
+                          int32_t heads, float scale, AttnPlan* plan);
+
+// Flash attention over the packed buffer. `pdl` marks the launch as a
+// programmatic dependent of the previous kernel on the stream.
+cudaError_t launch_attn_fwd(const AttnPlan& plan, cudaStream_t stream, bool pdl);
+
+// Synchronises the stream, then reads and clears the attention kernel's
+// device error word.
+cudaError_t read_and_clear_device_error(cudaStream_t stream, int32_t* code);
+
+}  // namespace wan

@@ -15,8 +15,21 @@
 // of the row in registers, so the row is read once, reduced (warp shuffles,
 // then one shared-memory exchange between the two warps), and written once.
 // The vector stride is 512 elements = 4 heads, so every vector of a thread
-// sits at the same head offset 8*(u%16): a thread needs the sines and cosines
-// of only 4 pairs per token, computed once per row.
+// sits at the same head offset 8*(u%16) and needs the rotations of only 4
+// pairs per token.
+//
+// Precision: the result is meant to be the correctly rounded value of the
+// definition, so that it matches an exact evaluation to 1 bf16 ulp everywhere
+// (a flipped rounding of y is amplified by a later near-cancelling rotation).
+//  - sum of squares in fp64 (bf16 values convert to doubles by bit moves);
+//  - r kept as a float pair r_hi + r_lo; y = round(x*g*r) is decided from
+//    v_hi = fl(x*g*r_hi), and recomputed exactly (sign of x*g*r - midpoint,
+//    with two FMAs) for the rare threads whose v_hi lies within 2 fp32 ulps
+//    of a bf16 rounding midpoint;
+//  - cos/sin from one fp64 sincos per thread (shared through shared memory),
+//    split as a 16-significant-bit head plus a float tail: the products of
+//    the 8-bit y with the heads are exact in fp32, so the rotation's only
+//    rounding is in the final sums.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -47,16 +60,13 @@ struct NormRopeParams {
   int32_t S, H, W;
   int32_t D;     // heads * 128
   int32_t nvec;  // D / 8 sixteen-byte vectors per row
-  float eps;
-  float inv_d;
-  float freq_over_pi[kPairs];  // per pair of a head: theta^(-2j/d_axis) / pi
+  double eps;
+  double inv_d;
+  double freq[kPairs];  // per pair of a head: theta^(-2j/d_axis)
 };
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-__device__ __forceinline__ float round_bf16(float x) {
-  return __bfloat162float(__float2bfloat16_rn(x));
-}
 
 __device__ __forceinline__ uint4 ld_stream(const uint16_t* p) {
   uint4 v;
@@ -74,28 +84,59 @@ __device__ __forceinline__ void st_v4(uint16_t* p, uint4 v) {
                : "memory");
 }
 
-__device__ __forceinline__ float sumsq(uint32_t w) {
-  float a = bf16_lo(w), b = bf16_hi(w);
-  return fmaf(a, a, b * b);
+// x^2 of both bf16 halves of w accumulated in fp64. A bf16 value's double has
+// the high word ((f32 bits >> 3) & 0x0FFFFFFF) + ((1023-127) << 20) and a zero
+// low word (the sign is dropped, irrelevant for a square; zero and subnormal
+// inputs map to ~2^-127, whose square is below 1e-76).
+__device__ __forceinline__ void sumsq_f64(uint32_t w, double& acc) {
+  const uint32_t hi_lo = ((w << 13) & 0x0FFFE000u) + 0x38000000u;
+  const uint32_t hi_hi = ((w >> 3) & 0x0FFFE000u) + 0x38000000u;
+  const double a = __hiloint2double(static_cast<int>(hi_lo), 0);
+  const double b = __hiloint2double(static_cast<int>(hi_hi), 0);
+  acc = fma(a, a, acc);
+  acc = fma(b, b, acc);
 }
 
-// One 32-bit word = one pair (x0 in the low half, x1 in the high half).
-__device__ __forceinline__ uint32_t norm_rotate_pair(uint32_t xw, uint32_t gw, float r, float c,
-                                                     float s) {
-  const float y0 = round_bf16(bf16_lo(xw) * r * bf16_lo(gw));
-  const float y1 = round_bf16(bf16_hi(xw) * r * bf16_hi(gw));
-  const float o0 = y0 * c - y1 * s;
-  const float o1 = y0 * s + y1 * c;
+// Distance (in fp32 ulps, mod 2^16) of v's low 16 bits from 0x7FFE: values
+// 0..4 mean v is within 2 ulps of a bf16 rounding midpoint.
+__device__ __forceinline__ uint32_t near_midpoint(float v) {
+  return (__float_as_uint(v) - 0x7FFEu) & 0xFFFFu;
+}
+
+// Correctly rounded bf16 (as 16 bits) of xg * (r_hi + r_lo), given
+// v_hi = fl(xg * r_hi): compares the exact product with the midpoint M above
+// v_hi's truncation using two FMAs (the sign of the result is exact).
+__device__ __forceinline__ uint32_t round_exact(float xg, float r_hi, float r_lo) {
+  const float v_hi = xg * r_hi;
+  const uint32_t t = __float_as_uint(v_hi) >> 16;  // truncation toward zero (sign-magnitude)
+  const float m = __uint_as_float((t << 16) | 0x8000u);
+  const float d = fmaf(xg, r_lo, fmaf(xg, r_hi, -m));
+  uint32_t up;
+  if (d == 0.f) {
+    up = t & 1u;  // exact tie: to even
+  } else {
+    up = ((__float_as_uint(d) ^ __float_as_uint(xg)) >> 31) ^ 1u;  // |v| beyond |M|
+  }
+  return (t + up) & 0xFFFFu;
+}
+
+// Rotation of one pair with the float-pair cos/sin (c = ch + cl, s = sh + sl).
+__device__ __forceinline__ uint32_t rotate_pair(uint32_t yw, const float4& cs) {
+  const float y0 = bf16_lo(yw), y1 = bf16_hi(yw);
+  const float o0 = fmaf(y0, cs.x, -(y1 * cs.z)) + fmaf(y0, cs.y, -(y1 * cs.w));
+  const float o1 = fmaf(y0, cs.z, y1 * cs.x) + fmaf(y0, cs.w, y1 * cs.y);
   return wan::sm100::pack_bf16x2(o0, o1);
 }
 
 template <int VPL>
 __global__ void __launch_bounds__(kThreads, 2) qk_norm_rope_kernel(const __grid_constant__ NormRopeParams p) {
-  __shared__ float partial[kRowsPerBlock * kWarpsPerRow];
+  __shared__ double partial[kRowsPerBlock * kWarpsPerRow];
+  __shared__ float4 rot[kRowsPerBlock][kPairs];  // (cos head, cos tail, sin head, sin tail)
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
-  const int u = threadIdx.x % kRowThreads;  // thread index within the row's warp pair
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * kRowsPerBlock + threadIdx.x / kRowThreads;
+  const int rib = threadIdx.x / kRowThreads;  // row in block
+  const int u = threadIdx.x % kRowThreads;    // thread index within the row's warp pair
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * kRowsPerBlock + rib;
   const bool active = row < p.rows;
   const int64_t tok = row >> 1;
   const int which = static_cast<int>(row & 1);  // 0: Q, 1: K
@@ -103,49 +144,79 @@ __global__ void __launch_bounds__(kThreads, 2) qk_norm_rope_kernel(const __grid_
   const uint16_t* g = which ? p.gamma_k : p.gamma_q;
 
   uint4 v[VPL];
-  float ss = 0.f;
 #pragma unroll
   for (int k = 0; k < VPL; ++k) {
     const int vi = u + kRowThreads * k;
     v[k] = (active && vi < p.nvec) ? ld_stream(x + 8 * vi) : make_uint4(0, 0, 0, 0);
   }
+
+  // This thread's share of the token's rotations: pair 4*(u%16) + u/16.
+  {
+    const int s = active ? static_cast<int>(tok % p.S) : 0;
+    const int pr = 4 * (u & 15) + (u >> 4);
+    const int pos = pr < kRowAxisPair0 ? s / (p.H * p.W)
+                                       : (pr < kColAxisPair0 ? (s / p.W) % p.H : s % p.W);
+    double sd, cd;
+    sincos(static_cast<double>(pos) * p.freq[pr], &sd, &cd);
+    const float ch = __uint_as_float(__float_as_uint(static_cast<float>(cd)) & 0xFFFFFF00u);
+    const float sh = __uint_as_float(__float_as_uint(static_cast<float>(sd)) & 0xFFFFFF00u);
+    rot[rib][pr] = make_float4(ch, static_cast<float>(cd - static_cast<double>(ch)), sh,
+                               static_cast<float>(sd - static_cast<double>(sh)));
+  }
+
+  double acc0 = 0.0, acc1 = 0.0, acc2 = 0.0, acc3 = 0.0;
 #pragma unroll
   for (int k = 0; k < VPL; ++k) {
-    ss += sumsq(v[k].x) + sumsq(v[k].y) + sumsq(v[k].z) + sumsq(v[k].w);
+    sumsq_f64(v[k].x, acc0);
+    sumsq_f64(v[k].y, acc1);
+    sumsq_f64(v[k].z, acc2);
+    sumsq_f64(v[k].w, acc3);
   }
+  double ss = (acc0 + acc1) + (acc2 + acc3);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
   if (lane == 0) partial[warp] = ss;
   __syncthreads();
-  const int w0 = (warp / kWarpsPerRow) * kWarpsPerRow;
-  const float total = partial[w0] + partial[w0 + 1];
-  const float r = 1.0f / sqrtf(total * p.inv_d + p.eps);
+  const int w0 = rib * kWarpsPerRow;
+  const double rd = 1.0 / sqrt((partial[w0] + partial[w0 + 1]) * p.inv_d + p.eps);
+  const float r_hi = static_cast<float>(rd);
+  const float r_lo = static_cast<float>(rd - static_cast<double>(r_hi));
 
   if (active) {
-    // Grid position of the token (width fastest) and this thread's 4 rotations.
-    const int s = static_cast<int>(tok % p.S);
-    const int hw = p.H * p.W;
-    const int pos_f = s / hw;
-    const int pos_h = (s / p.W) % p.H;
-    const int pos_w = s % p.W;
     const int pair0 = (u & 15) * 4;
-    float cs[4], sn[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int pr = pair0 + i;
-      const int pos = pr < kRowAxisPair0 ? pos_f : (pr < kColAxisPair0 ? pos_h : pos_w);
-      sincospif(static_cast<float>(pos) * p.freq_over_pi[pr], &sn[i], &cs[i]);
-    }
+    const float4 cs0 = rot[rib][pair0], cs1 = rot[rib][pair0 + 1];
+    const float4 cs2 = rot[rib][pair0 + 2], cs3 = rot[rib][pair0 + 3];
 #pragma unroll
     for (int k = 0; k < VPL; ++k) {
       const int vi = u + kRowThreads * k;
       if (vi < p.nvec) {
         const uint4 gv = ld_cached(g + 8 * vi);
+        const uint32_t xw[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+        const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+        uint32_t yw[4];
+        uint32_t near = 0xFFFFu;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float xg0 = bf16_lo(xw[e]) * bf16_lo(gw[e]);  // exact: 8-bit x 8-bit significands
+          const float xg1 = bf16_hi(xw[e]) * bf16_hi(gw[e]);
+          const float v0 = xg0 * r_hi, v1 = xg1 * r_hi;
+          near = min(near, min(near_midpoint(v0), near_midpoint(v1)));
+          yw[e] = wan::sm100::pack_bf16x2(v0, v1);
+        }
+        if (near <= 4u) {
+          // Rare: some v_hi is within 2 ulps of a rounding midpoint.
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const uint32_t lo = round_exact(bf16_lo(xw[e]) * bf16_lo(gw[e]), r_hi, r_lo);
+            const uint32_t hi = round_exact(bf16_hi(xw[e]) * bf16_hi(gw[e]), r_hi, r_lo);
+            yw[e] = lo | (hi << 16);
+          }
+        }
         uint4 o;
-        o.x = norm_rotate_pair(v[k].x, gv.x, r, cs[0], sn[0]);
-        o.y = norm_rotate_pair(v[k].y, gv.y, r, cs[1], sn[1]);
-        o.z = norm_rotate_pair(v[k].z, gv.z, r, cs[2], sn[2]);
-        o.w = norm_rotate_pair(v[k].w, gv.w, r, cs[3], sn[3]);
+        o.x = rotate_pair(yw[0], cs0);
+        o.y = rotate_pair(yw[1], cs1);
+        o.z = rotate_pair(yw[2], cs2);
+        o.w = rotate_pair(yw[3], cs3);
         st_v4(x + 8 * vi, o);
       }
     }
@@ -177,14 +248,13 @@ cudaError_t launch_qk_norm_rope(void* qkv, int64_t batch, int32_t F, int32_t H, 
   p.D = heads * kHeadDim;
   p.nvec = p.D / 8;
   p.rows = batch * static_cast<int64_t>(p.S) * 2;
-  p.eps = eps;
-  p.inv_d = 1.0f / static_cast<float>(p.D);
+  p.eps = static_cast<double>(eps);
+  p.inv_d = 1.0 / static_cast<double>(p.D);
   const int split[3] = {44, 42, 42};
   for (int pr = 0; pr < kPairs; ++pr) {
     const int axis = pr < kRowAxisPair0 ? 0 : (pr < kColAxisPair0 ? 1 : 2);
     const int j = pr - (axis == 0 ? 0 : (axis == 1 ? kRowAxisPair0 : kColAxisPair0));
-    p.freq_over_pi[pr] = static_cast<float>(
-        std::pow(static_cast<double>(theta), -2.0 * j / static_cast<double>(split[axis])) / M_PI);
+    p.freq[pr] = std::pow(static_cast<double>(theta), -2.0 * j / static_cast<double>(split[axis]));
   }
   if (p.rows == 0) return cudaSuccess;
   const int vpl = (p.nvec + kRowThreads - 1) / kRowThreads;  // 16-byte vectors per thread

@@ -48,8 +48,8 @@ NORM_SRC = os.path.join(ROOT, "video_diffusion_transformer_packed_b200", "csrc",
 def parse_args():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
-    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=wi.BENCH_WORKLOAD.name, choices=sorted(wi.BY_NAME))
     ap.add_argument("--cpu-seconds", type=float, default=12.0,

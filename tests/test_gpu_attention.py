@@ -53,8 +53,7 @@ def test_batches_do_not_leak():
     """Two batches with different content; rows past S in the last tile must
     read as zeros of the same batch, not the next batch's tokens."""
     S, heads = 200, 3
-    qkv = wi.packed_qkv(2, S, heads, seed=3)
-    qkv[1] = (qkv[1].float() * 2.0).to(torch.bfloat16)
+    qkv = torch.cat([wi.packed_qkv(1, S, heads, seed=3), wi.packed_qkv(1, S, heads, seed=33)])
     got = gpu_attention(qkv, heads)
     ref = oracle.attention_full(qkv, heads, SCALE)
     assert_attention_close(got.view(2, S, heads, HD), ref, "batch")
@@ -69,7 +68,7 @@ def test_peaked_logits_force_rescaling():
     qkv = qkv.to(torch.bfloat16)
     got = gpu_attention(qkv, heads)
     ref = oracle.attention_full(qkv, heads, SCALE)
-    assert_attention_close(got.view(1, S, heads, HD), ref, "peaked")
+    assert_attention_close(got.view(1, S, heads, HD), ref, "peaked", scaled=True)
 
 
 def test_large_scale_spread_logits():
@@ -77,7 +76,7 @@ def test_large_scale_spread_logits():
     qkv = wi.packed_qkv(1, S, heads, seed=5)
     got = gpu_attention(qkv, heads, scale=0.5)
     ref = oracle.attention_full(qkv, heads, 0.5)
-    assert_attention_close(got.view(1, S, heads, HD), ref, "scale 0.5")
+    assert_attention_close(got.view(1, S, heads, HD), ref, "scale 0.5", scaled=True)
 
 
 def test_constant_v_gives_v():

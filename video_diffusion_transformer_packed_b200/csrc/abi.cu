@@ -167,9 +167,12 @@ int32_t wan_dit_attn(void* qkv, void* out, int64_t batch, int32_t F, int32_t H, 
 int32_t wan_device_error(void* stream, int32_t* code) {
   if (!code) return WAN_ERR_NULL;
   *code = 0;
-  if (wan::read_and_clear_device_error(static_cast<cudaStream_t>(stream), code) != cudaSuccess) {
+  int32_t attn = 0, norm = 0;
+  if (wan::read_and_clear_device_error(static_cast<cudaStream_t>(stream), &attn) != cudaSuccess ||
+      wan::read_and_clear_norm_error(static_cast<cudaStream_t>(stream), &norm) != cudaSuccess) {
     return WAN_ERR_LAUNCH;
   }
+  *code = attn | (norm << 8);
   return *code != 0 ? WAN_ERR_DEVICE_TIMEOUT : WAN_OK;
 }
 

@@ -10,13 +10,17 @@
 // with head dims [0,44) on the frame axis, [44,86) on rows, [86,128) on columns.
 //
 // Design: the op is HBM-bound (read + write of Q and K once: 8*D bytes per
-// token, V untouched). Two warps own one (token, Q-or-K) row of D elements:
-// thread u (0..63) of the pair holds the 16-byte vectors u, u+64, u+128, ...
-// of the row in registers, so the row is read once, reduced (warp shuffles,
-// then one shared-memory exchange between the two warps), and written once.
-// The vector stride is 512 elements = 4 heads, so every vector of a thread
-// sits at the same head offset 8*(u%16) and needs the rotations of only 4
-// pairs per token.
+// token, V untouched). A persistent grid (a few CTAs per SM) walks the tokens.
+// A token's Q and K rows are contiguous in the packed buffer, so one bulk
+// copy (cp.async.bulk, the untiled TMA) stages both into a shared-memory
+// ring several tokens ahead of the threads that consume them; the reads of
+// the next tokens are in flight while the current one is computed. Warps 0-3
+// take the Q row, warps 4-7 the K row: thread u (0..127) of a row holds the
+// 16-byte vectors u, u+128, ... in registers, the row's sum of squares is
+// reduced with warp shuffles and one shared-memory exchange, and results go
+// straight to global memory with 16-byte stores (in place). The vector
+// stride (1024 elements = 8 heads) keeps every vector of a thread at the
+// same head offset 8*(u%16), so a thread needs the rotations of 4 pairs.
 //
 // Precision: the result is meant to be the correctly rounded value of the
 // definition, so that it matches an exact evaluation to 1 bf16 ulp everywhere
@@ -44,35 +48,48 @@ namespace {
 
 constexpr int kHeadDim = 128;
 constexpr int kPairs = kHeadDim / 2;
-constexpr int kWarpsPerRow = 2;
-constexpr int kRowThreads = 32 * kWarpsPerRow;
-constexpr int kRowsPerBlock = 4;
-constexpr int kThreads = kRowThreads * kRowsPerBlock;
+constexpr int kThreads = 256;    // warps 0-3: the Q row of a token, warps 4-7: its K row
+constexpr int kRowThreads = 128;
+constexpr int kMaxStages = 8;
+constexpr uint32_t kStageBudget = 72 * 1024;  // ring bytes per CTA (3 CTAs fit an SM)
+constexpr uint64_t kWaitLimitNs = 1000000000ull;
 // Pair index where the row axis and the column axis start (split 44/42/42).
 constexpr int kRowAxisPair0 = 44 / 2;
 constexpr int kColAxisPair0 = (44 + 42) / 2;
+
+__device__ int g_norm_error_word;
 
 struct NormRopeParams {
   uint16_t* qkv;
   const uint16_t* gamma_q;
   const uint16_t* gamma_k;
-  int64_t rows;  // batch * S * 2 (Q and K rows of each token)
+  int64_t tokens;        // batch * S
   int32_t S, H, W;
-  int32_t D;     // heads * 128
-  int32_t nvec;  // D / 8 sixteen-byte vectors per row
+  int32_t D;             // heads * 128
+  int32_t nvec;          // D / 8 sixteen-byte vectors per row
+  int32_t stages;        // ring depth
+  uint32_t stage_bytes;  // Q row + K row = 4 * D bytes
   double eps;
   double inv_d;
-  double freq[kPairs];  // per pair of a head: theta^(-2j/d_axis)
+  double freq[kPairs];   // per pair of a head: theta^(-2j/d_axis)
+};
+
+// Shared-memory layout behind the ring (offsets from the ring's end).
+struct alignas(16) NormSmemTail {
+  uint64_t full[kMaxStages];
+  double partial[2][8];            // per warp sums of squares, double-buffered by token parity
+  float4 rot[2][kPairs];           // (cos head, cos tail, sin head, sin tail) per pair
+  int abort;
 };
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-__device__ __forceinline__ uint4 ld_stream(const uint16_t* p) {
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
   uint4 v;
-  asm volatile("ld.global.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
+               : "r"(addr));
   return v;
 }
 __device__ __forceinline__ uint4 ld_cached(const uint16_t* p) {
@@ -128,66 +145,115 @@ __device__ __forceinline__ uint32_t rotate_pair(uint32_t yw, const float4& cs) {
   return wan::sm100::pack_bf16x2(o0, o1);
 }
 
-template <int VPL>
-__global__ void __launch_bounds__(kThreads, 2) qk_norm_rope_kernel(const __grid_constant__ NormRopeParams p) {
-  __shared__ double partial[kRowsPerBlock * kWarpsPerRow];
-  __shared__ float4 rot[kRowsPerBlock][kPairs];  // (cos head, cos tail, sin head, sin tail)
-  const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
-  const int rib = threadIdx.x / kRowThreads;  // row in block
-  const int u = threadIdx.x % kRowThreads;    // thread index within the row's warp pair
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * kRowsPerBlock + rib;
-  const bool active = row < p.rows;
-  const int64_t tok = row >> 1;
-  const int which = static_cast<int>(row & 1);  // 0: Q, 1: K
-  uint16_t* x = p.qkv + tok * 3 * static_cast<int64_t>(p.D) + which * p.D;
-  const uint16_t* g = which ? p.gamma_k : p.gamma_q;
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
 
-  uint4 v[VPL];
-#pragma unroll
-  for (int k = 0; k < VPL; ++k) {
-    const int vi = u + kRowThreads * k;
-    v[k] = (active && vi < p.nvec) ? ld_stream(x + 8 * vi) : make_uint4(0, 0, 0, 0);
-  }
+template <int VPT>
+__global__ void __launch_bounds__(kThreads) qk_norm_rope_kernel(const __grid_constant__ NormRopeParams p) {
+  using namespace wan::sm100;
+  extern __shared__ __align__(128) uint8_t smem[];
+  NormSmemTail& tail = *reinterpret_cast<NormSmemTail*>(smem + p.stages * p.stage_bytes);
+  const uint32_t ring = smem_u32(smem);
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+  const int which = warp >> 2;  // 0: Q, 1: K
+  const int u = tid & (kRowThreads - 1);
+  const int64_t step = gridDim.x;
 
-  // This thread's share of the token's rotations: pair 4*(u%16) + u/16.
-  {
-    const int s = active ? static_cast<int>(tok % p.S) : 0;
-    const int pr = 4 * (u & 15) + (u >> 4);
-    const int pos = pr < kRowAxisPair0 ? s / (p.H * p.W)
-                                       : (pr < kColAxisPair0 ? (s / p.W) % p.H : s % p.W);
-    double sd, cd;
-    sincos(static_cast<double>(pos) * p.freq[pr], &sd, &cd);
-    const float ch = __uint_as_float(__float_as_uint(static_cast<float>(cd)) & 0xFFFFFF00u);
-    const float sh = __uint_as_float(__float_as_uint(static_cast<float>(sd)) & 0xFFFFFF00u);
-    rot[rib][pr] = make_float4(ch, static_cast<float>(cd - static_cast<double>(ch)), sh,
-                               static_cast<float>(sd - static_cast<double>(sh)));
+  if (tid == 0) {
+    for (int s = 0; s < p.stages; ++s) mbar_init(smem_u32(&tail.full[s]), 1);
+    tail.abort = 0;
+    fence_mbar_init();
   }
-
-  double acc0 = 0.0, acc1 = 0.0, acc2 = 0.0, acc3 = 0.0;
-#pragma unroll
-  for (int k = 0; k < VPL; ++k) {
-    sumsq_f64(v[k].x, acc0);
-    sumsq_f64(v[k].y, acc1);
-    sumsq_f64(v[k].z, acc2);
-    sumsq_f64(v[k].w, acc3);
-  }
-  double ss = (acc0 + acc1) + (acc2 + acc3);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  if (lane == 0) partial[warp] = ss;
   __syncthreads();
-  const int w0 = rib * kWarpsPerRow;
-  const double rd = 1.0 / sqrt((partial[w0] + partial[w0 + 1]) * p.inv_d + p.eps);
-  const float r_hi = static_cast<float>(rd);
-  const float r_lo = static_cast<float>(rd - static_cast<double>(r_hi));
+  int64_t n_issued = 0;  // copies started (thread 0 only): iterations 0 .. n_issued-1
+  if (tid == 0) {
+    for (int s = 0; s < p.stages; ++s) {
+      const int64_t tok = blockIdx.x + s * step;
+      if (tok < p.tokens) {
+        const uint32_t bar = smem_u32(&tail.full[s]);
+        mbar_arrive_expect_tx(bar, p.stage_bytes);
+        bulk_load(ring + s * p.stage_bytes, p.qkv + tok * 3 * static_cast<int64_t>(p.D), p.stage_bytes, bar);
+        ++n_issued;
+      }
+    }
+  }
 
-  if (active) {
-    const int pair0 = (u & 15) * 4;
-    const float4 cs0 = rot[rib][pair0], cs1 = rot[rib][pair0 + 1];
-    const float4 cs2 = rot[rib][pair0 + 2], cs3 = rot[rib][pair0 + 3];
+  int64_t i = 0;
+  for (int64_t tok = blockIdx.x; tok < p.tokens; tok += step, ++i) {
+    const int stage = static_cast<int>(i % p.stages);
+    const uint32_t parity = static_cast<uint32_t>((i / p.stages) & 1);
+    const int buf = static_cast<int>(i & 1);
+    if (!mbar_wait(smem_u32(&tail.full[stage]), parity, nullptr, kWaitLimitNs)) {
+      tail.abort = 1;
+      atomicOr(&g_norm_error_word, 1);
+    }
+
+    // This row's vectors, out of the staged token.
+    const uint32_t src = ring + stage * p.stage_bytes + which * p.D * 2;
+    uint4 v[VPT];
 #pragma unroll
-    for (int k = 0; k < VPL; ++k) {
+    for (int k = 0; k < VPT; ++k) {
+      const int vi = u + kRowThreads * k;
+      v[k] = vi < p.nvec ? ld_shared_v4(src + 16 * vi) : make_uint4(0, 0, 0, 0);
+    }
+
+    // The token's 64 rotations: one fp64 sincos on every 4th thread.
+    const int s = static_cast<int>(tok % p.S);
+    if ((tid & 3) == 0) {
+      const int pr = tid >> 2;
+      const int pos = pr < kRowAxisPair0 ? s / (p.H * p.W)
+                                         : (pr < kColAxisPair0 ? (s / p.W) % p.H : s % p.W);
+      double sd, cd;
+      sincos(static_cast<double>(pos) * p.freq[pr], &sd, &cd);
+      const float ch = __uint_as_float(__float_as_uint(static_cast<float>(cd)) & 0xFFFFFF00u);
+      const float sh = __uint_as_float(__float_as_uint(static_cast<float>(sd)) & 0xFFFFFF00u);
+      tail.rot[buf][pr] = make_float4(ch, static_cast<float>(cd - static_cast<double>(ch)), sh,
+                                      static_cast<float>(sd - static_cast<double>(sh)));
+    }
+
+    double acc0 = 0.0, acc1 = 0.0, acc2 = 0.0, acc3 = 0.0;
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) {
+      sumsq_f64(v[k].x, acc0);
+      sumsq_f64(v[k].y, acc1);
+      sumsq_f64(v[k].z, acc2);
+      sumsq_f64(v[k].w, acc3);
+    }
+    double ss = (acc0 + acc1) + (acc2 + acc3);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (lane == 0) tail.partial[buf][warp] = ss;
+    __syncthreads();  // the stage is consumed; partial sums and rotations are visible
+    if (tail.abort) break;
+
+    if (tid == 0) {
+      const int64_t next = tok + p.stages * step;
+      if (next < p.tokens) {
+        const uint32_t bar = smem_u32(&tail.full[stage]);
+        mbar_arrive_expect_tx(bar, p.stage_bytes);
+        bulk_load(ring + stage * p.stage_bytes, p.qkv + next * 3 * static_cast<int64_t>(p.D),
+                  p.stage_bytes, bar);
+        ++n_issued;
+      }
+    }
+
+    const double* part = &tail.partial[buf][4 * which];
+    const double rd = 1.0 / sqrt(((part[0] + part[1]) + (part[2] + part[3])) * p.inv_d + p.eps);
+    const float r_hi = static_cast<float>(rd);
+    const float r_lo = static_cast<float>(rd - static_cast<double>(r_hi));
+    const int pair0 = (u & 15) * 4;
+    const float4 cs0 = tail.rot[buf][pair0], cs1 = tail.rot[buf][pair0 + 1];
+    const float4 cs2 = tail.rot[buf][pair0 + 2], cs3 = tail.rot[buf][pair0 + 3];
+    const uint16_t* g = which ? p.gamma_k : p.gamma_q;
+    uint16_t* x = p.qkv + tok * 3 * static_cast<int64_t>(p.D) + which * p.D;
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) {
       const int vi = u + kRowThreads * k;
       if (vi < p.nvec) {
         const uint4 gv = ld_cached(g + 8 * vi);
@@ -201,7 +267,7 @@ __global__ void __launch_bounds__(kThreads, 2) qk_norm_rope_kernel(const __grid_
           const float xg1 = bf16_hi(xw[e]) * bf16_hi(gw[e]);
           const float v0 = xg0 * r_hi, v1 = xg1 * r_hi;
           near = min(near, min(near_midpoint(v0), near_midpoint(v1)));
-          yw[e] = wan::sm100::pack_bf16x2(v0, v1);
+          yw[e] = pack_bf16x2(v0, v1);
         }
         if (near <= 4u) {
           // Rare: some v_hi is within 2 ulps of a rounding midpoint.
@@ -221,15 +287,41 @@ __global__ void __launch_bounds__(kThreads, 2) qk_norm_rope_kernel(const __grid_
       }
     }
   }
+  if (tail.abort && tid == 0) {
+    // Let every copy this block started land before it exits.
+    for (int s2 = 0; s2 < p.stages; ++s2) {
+      const int64_t uses = n_issued > s2 ? (n_issued - s2 + p.stages - 1) / p.stages : 0;
+      if (uses > 0) {
+        mbar_wait(smem_u32(&tail.full[s2]), static_cast<uint32_t>((uses - 1) & 1), nullptr, kWaitLimitNs);
+      }
+    }
+  }
   // Let a programmatically dependent launch (the attention kernel) start its
   // prologue; it still waits for this grid's completion before reading.
-  wan::sm100::grid_launch_dependents();
+  grid_launch_dependents();
 }
 
-template <int VPL>
-cudaError_t launch_vpl(const NormRopeParams& p, cudaStream_t stream) {
-  const int64_t blocks = (p.rows + kRowsPerBlock - 1) / kRowsPerBlock;
-  qk_norm_rope_kernel<VPL><<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(p);
+template <int VPT>
+cudaError_t launch_vpt(const NormRopeParams& p, uint32_t smem_bytes, cudaStream_t stream) {
+  static int blocks_per_sm = -1;  // per instantiation; the smem size is fixed per instantiation
+  static uint32_t configured_smem = 0;
+  if (configured_smem != smem_bytes) {
+    cudaError_t e = cudaFuncSetAttribute(qk_norm_rope_kernel<VPT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem_bytes));
+    if (e != cudaSuccess) return e;
+    int n = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, qk_norm_rope_kernel<VPT>, kThreads, smem_bytes);
+    if (e != cudaSuccess) return e;
+    blocks_per_sm = n > 0 ? n : 1;
+    configured_smem = smem_bytes;
+  }
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  const int64_t want = static_cast<int64_t>(sms) * blocks_per_sm;
+  const int64_t blocks = p.tokens < want ? p.tokens : want;
+  qk_norm_rope_kernel<VPT><<<static_cast<unsigned>(blocks), kThreads, smem_bytes, stream>>>(p);
   return cudaGetLastError();
 }
 
@@ -247,7 +339,10 @@ cudaError_t launch_qk_norm_rope(void* qkv, int64_t batch, int32_t F, int32_t H, 
   p.W = W;
   p.D = heads * kHeadDim;
   p.nvec = p.D / 8;
-  p.rows = batch * static_cast<int64_t>(p.S) * 2;
+  p.tokens = batch * static_cast<int64_t>(p.S);
+  p.stage_bytes = 4u * static_cast<uint32_t>(p.D);
+  int stages = static_cast<int>(kStageBudget / p.stage_bytes);
+  p.stages = stages < 2 ? 2 : (stages > kMaxStages ? kMaxStages : stages);
   p.eps = static_cast<double>(eps);
   p.inv_d = 1.0 / static_cast<double>(p.D);
   const int split[3] = {44, 42, 42};
@@ -256,17 +351,34 @@ cudaError_t launch_qk_norm_rope(void* qkv, int64_t batch, int32_t F, int32_t H, 
     const int j = pr - (axis == 0 ? 0 : (axis == 1 ? kRowAxisPair0 : kColAxisPair0));
     p.freq[pr] = std::pow(static_cast<double>(theta), -2.0 * j / static_cast<double>(split[axis]));
   }
-  if (p.rows == 0) return cudaSuccess;
-  const int vpl = (p.nvec + kRowThreads - 1) / kRowThreads;  // 16-byte vectors per thread
-  if (vpl <= 1) return launch_vpl<1>(p, stream);
-  if (vpl <= 2) return launch_vpl<2>(p, stream);
-  if (vpl <= 3) return launch_vpl<3>(p, stream);
-  if (vpl <= 4) return launch_vpl<4>(p, stream);
-  if (vpl <= 6) return launch_vpl<6>(p, stream);
-  if (vpl <= 8) return launch_vpl<8>(p, stream);
-  if (vpl <= 10) return launch_vpl<10>(p, stream);
-  if (vpl <= 12) return launch_vpl<12>(p, stream);
-  return launch_vpl<16>(p, stream);
+  if (p.tokens == 0) return cudaSuccess;
+  const uint32_t smem_bytes = p.stages * p.stage_bytes + static_cast<uint32_t>(sizeof(NormSmemTail));
+  const int vpt = (p.nvec + kRowThreads - 1) / kRowThreads;  // 16-byte vectors per thread
+  switch (vpt) {
+    case 1: return launch_vpt<1>(p, smem_bytes, stream);
+    case 2: return launch_vpt<2>(p, smem_bytes, stream);
+    case 3: return launch_vpt<3>(p, smem_bytes, stream);
+    case 4: return launch_vpt<4>(p, smem_bytes, stream);
+    case 5: return launch_vpt<5>(p, smem_bytes, stream);
+    case 6: return launch_vpt<6>(p, smem_bytes, stream);
+    case 7: return launch_vpt<7>(p, smem_bytes, stream);
+    default: return launch_vpt<8>(p, smem_bytes, stream);
+  }
+}
+
+cudaError_t read_and_clear_norm_error(cudaStream_t stream, int32_t* code) {
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return e;
+  int v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_norm_error_word, sizeof(int));
+  if (e != cudaSuccess) return e;
+  if (v != 0) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(g_norm_error_word, &zero, sizeof(int));
+    if (e != cudaSuccess) return e;
+  }
+  *code = v;
+  return cudaSuccess;
 }
 
 }  // namespace wan

@@ -31,8 +31,8 @@ cudaError_t plan_attn_fwd(const void* qkv, void* out, int64_t batch, int64_t seq
 // programmatic dependent of the previous kernel on the stream.
 cudaError_t launch_attn_fwd(const AttnPlan& plan, cudaStream_t stream, bool pdl);
 
-// Synchronises the stream, then reads and clears the attention kernel's
-// device error word.
+// Synchronise the stream, then read and clear a kernel's device error word.
 cudaError_t read_and_clear_device_error(cudaStream_t stream, int32_t* code);
+cudaError_t read_and_clear_norm_error(cudaStream_t stream, int32_t* code);
 
 }  // namespace wan

@@ -78,7 +78,9 @@ struct NormRopeParams {
 struct alignas(16) NormSmemTail {
   uint64_t full[kMaxStages];
   double partial[2][8];            // per warp sums of squares, double-buffered by token parity
-  float4 rot[2][kPairs];           // (cos head, cos tail, sin head, sin tail) per pair
+  float4 rot[3][kPairs][2];        // per pair: (ch, sh, -sh, ch), (cl, sl, -sl, cl) -- cos/sin
+                                   // heads and tails as f32x2 operands; the table of
+                                   // iteration i+1 is written during iteration i
   int abort;
 };
 
@@ -101,25 +103,6 @@ __device__ __forceinline__ void st_v4(uint16_t* p, uint4 v) {
                : "memory");
 }
 
-// x^2 of both bf16 halves of w accumulated in fp64. A bf16 value's double has
-// the high word ((f32 bits >> 3) & 0x0FFFFFFF) + ((1023-127) << 20) and a zero
-// low word (the sign is dropped, irrelevant for a square; zero and subnormal
-// inputs map to ~2^-127, whose square is below 1e-76).
-__device__ __forceinline__ void sumsq_f64(uint32_t w, double& acc) {
-  const uint32_t hi_lo = ((w << 13) & 0x0FFFE000u) + 0x38000000u;
-  const uint32_t hi_hi = ((w >> 3) & 0x0FFFE000u) + 0x38000000u;
-  const double a = __hiloint2double(static_cast<int>(hi_lo), 0);
-  const double b = __hiloint2double(static_cast<int>(hi_hi), 0);
-  acc = fma(a, a, acc);
-  acc = fma(b, b, acc);
-}
-
-// Distance (in fp32 ulps, mod 2^16) of v's low 16 bits from 0x7FFE: values
-// 0..4 mean v is within 2 ulps of a bf16 rounding midpoint.
-__device__ __forceinline__ uint32_t near_midpoint(float v) {
-  return (__float_as_uint(v) - 0x7FFEu) & 0xFFFFu;
-}
-
 // Correctly rounded bf16 (as 16 bits) of xg * (r_hi + r_lo), given
 // v_hi = fl(xg * r_hi): compares the exact product with the midpoint M above
 // v_hi's truncation using two FMAs (the sign of the result is exact).
@@ -137,14 +120,6 @@ __device__ __forceinline__ uint32_t round_exact(float xg, float r_hi, float r_lo
   return (t + up) & 0xFFFFu;
 }
 
-// Rotation of one pair with the float-pair cos/sin (c = ch + cl, s = sh + sl).
-__device__ __forceinline__ uint32_t rotate_pair(uint32_t yw, const float4& cs) {
-  const float y0 = bf16_lo(yw), y1 = bf16_hi(yw);
-  const float o0 = fmaf(y0, cs.x, -(y1 * cs.z)) + fmaf(y0, cs.y, -(y1 * cs.w));
-  const float o1 = fmaf(y0, cs.z, y1 * cs.x) + fmaf(y0, cs.w, y1 * cs.y);
-  return wan::sm100::pack_bf16x2(o0, o1);
-}
-
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
@@ -152,8 +127,83 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
       : "memory");
 }
 
+// Rotation table entries of pair `pr` for sequence index s (one fp64 sincos):
+// cos/sin split into a 16-significant-bit head and a float tail.
+__device__ __forceinline__ void rotation(const NormRopeParams& p, int s, int pr, float4* dst) {
+  const int q = s / p.W;  // frame * H + row
+  const int pos = pr < kRowAxisPair0 ? q / p.H : (pr < kColAxisPair0 ? q - (q / p.H) * p.H : s - q * p.W);
+  double sd, cd;
+  sincos(static_cast<double>(pos) * p.freq[pr], &sd, &cd);
+  const float ch = __uint_as_float(__float_as_uint(static_cast<float>(cd)) & 0xFFFFFF00u);
+  const float sh = __uint_as_float(__float_as_uint(static_cast<float>(sd)) & 0xFFFFFF00u);
+  const float cl = static_cast<float>(cd - static_cast<double>(ch));
+  const float sl = static_cast<float>(sd - static_cast<double>(sh));
+  dst[0] = make_float4(ch, sh, -sh, ch);
+  dst[1] = make_float4(cl, sl, -sl, cl);
+}
+
+// ---- packed fp32x2 arithmetic (one instruction for two lanes of a pair)
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1,%2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0,%1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+
+// x^2 of both bf16 halves of w accumulated in fp64. A bf16 value's double
+// has the high word ((f32 bits >> 3) & 0x0FFFFFFF) + ((1023-127) << 20) and a
+// zero low word (the sign is dropped, irrelevant for a square; zero and
+// subnormal inputs map to ~2^-127, whose square is below 1e-76).
+__device__ __forceinline__ void sumsq_pair(uint32_t w, double& acc_lo, double& acc_hi) {
+  const uint32_t hw_lo = (w & 0x7FFFu) * 8192u + 0x38000000u;
+  const uint32_t hw_hi = __umulhi(w & 0x7FFF0000u, 1u << 29) + 0x38000000u;
+  const double a = __hiloint2double(static_cast<int>(hw_lo), 0);
+  const double b = __hiloint2double(static_cast<int>(hw_hi), 0);
+  acc_lo = fma(a, a, acc_lo);
+  acc_hi = fma(b, b, acc_hi);
+}
+
+// One pair: v = x*g*r_hi (x*g is exact) rounded to bf16. `near` keeps the
+// per-16-bit-lane minimum of (low 16 bits of v) + 0x8002, which is below 8
+// when v lies within a few fp32 ulps of a bf16 rounding midpoint (a carry
+// from the low lane only widens the high lane's window).
+__device__ __forceinline__ uint32_t norm_round(uint32_t xw, uint32_t gw, uint64_t r2, uint32_t& near) {
+  const uint64_t x = f2(bf16_lo(xw), bf16_hi(xw));
+  const uint64_t g = f2(bf16_lo(gw), bf16_hi(gw));
+  const uint64_t v = mul2(mul2(x, g), r2);
+  float v0, v1;
+  f2_split(v, v0, v1);
+  const uint32_t lows = __byte_perm(__float_as_uint(v0), __float_as_uint(v1), 0x5410);
+  near = __vminu2(near, lows + 0x80028002u);
+  return wan::sm100::pack_bf16x2(v0, v1);
+}
+
+__device__ __forceinline__ uint32_t rotate(uint32_t yw, const float4& A, const float4& B) {
+  const float y0 = bf16_lo(yw), y1 = bf16_hi(yw);
+  const uint64_t yy0 = f2(y0, y0), yy1 = f2(y1, y1);
+  // (y0 ch - y1 sh, y0 sh + y1 ch): head products are exact, one rounding.
+  uint64_t o = fma2(yy0, f2(A.x, A.y), mul2(yy1, f2(A.z, A.w)));
+  o = fma2(yy1, f2(B.z, B.w), o);  // + (-y1 sl, y1 cl)
+  o = fma2(yy0, f2(B.x, B.y), o);  // + (y0 cl, y0 sl)
+  float o0, o1;
+  f2_split(o, o0, o1);
+  return wan::sm100::pack_bf16x2(o0, o1);
+}
+
 template <int VPT>
-__global__ void __launch_bounds__(kThreads) qk_norm_rope_kernel(const __grid_constant__ NormRopeParams p) {
+__global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const __grid_constant__ NormRopeParams p) {
   using namespace wan::sm100;
   extern __shared__ __align__(128) uint8_t smem[];
   NormSmemTail& tail = *reinterpret_cast<NormSmemTail*>(smem + p.stages * p.stage_bytes);
@@ -184,11 +234,25 @@ __global__ void __launch_bounds__(kThreads) qk_norm_rope_kernel(const __grid_con
     }
   }
 
+  const uint16_t* g = which ? p.gamma_k : p.gamma_q;
+
+  // Sequence index of the current token and of the next one, kept
+  // incrementally (no 64-bit division in the loop).
+  const int step_mod = static_cast<int>(step % p.S);
+  int s_next = static_cast<int>(blockIdx.x % p.S);
+  if ((tid & 3) == 0) rotation(p, s_next, tid >> 2, tail.rot[0][tid >> 2]);
+  s_next += step_mod;
+  if (s_next >= p.S) s_next -= p.S;
+  __syncthreads();
+
+  int stage = 0, rbuf = 0;
+  uint32_t parity = 0;
   int64_t i = 0;
   for (int64_t tok = blockIdx.x; tok < p.tokens; tok += step, ++i) {
-    const int stage = static_cast<int>(i % p.stages);
-    const uint32_t parity = static_cast<uint32_t>((i / p.stages) & 1);
     const int buf = static_cast<int>(i & 1);
+    // The next token's rotations, ahead of time (they do not depend on the data).
+    const int rnext = rbuf == 2 ? 0 : rbuf + 1;
+    if ((tid & 3) == 0 && tok + step < p.tokens) rotation(p, s_next, tid >> 2, tail.rot[rnext][tid >> 2]);
     if (!mbar_wait(smem_u32(&tail.full[stage]), parity, nullptr, kWaitLimitNs)) {
       tail.abort = 1;
       atomicOr(&g_norm_error_word, 1);
@@ -203,29 +267,15 @@ __global__ void __launch_bounds__(kThreads) qk_norm_rope_kernel(const __grid_con
       v[k] = vi < p.nvec ? ld_shared_v4(src + 16 * vi) : make_uint4(0, 0, 0, 0);
     }
 
-    // The token's 64 rotations: one fp64 sincos on every 4th thread.
-    const int s = static_cast<int>(tok % p.S);
-    if ((tid & 3) == 0) {
-      const int pr = tid >> 2;
-      const int pos = pr < kRowAxisPair0 ? s / (p.H * p.W)
-                                         : (pr < kColAxisPair0 ? (s / p.W) % p.H : s % p.W);
-      double sd, cd;
-      sincos(static_cast<double>(pos) * p.freq[pr], &sd, &cd);
-      const float ch = __uint_as_float(__float_as_uint(static_cast<float>(cd)) & 0xFFFFFF00u);
-      const float sh = __uint_as_float(__float_as_uint(static_cast<float>(sd)) & 0xFFFFFF00u);
-      tail.rot[buf][pr] = make_float4(ch, static_cast<float>(cd - static_cast<double>(ch)), sh,
-                                      static_cast<float>(sd - static_cast<double>(sh)));
-    }
-
-    double acc0 = 0.0, acc1 = 0.0, acc2 = 0.0, acc3 = 0.0;
+    double acc[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
 #pragma unroll
     for (int k = 0; k < VPT; ++k) {
-      sumsq_f64(v[k].x, acc0);
-      sumsq_f64(v[k].y, acc1);
-      sumsq_f64(v[k].z, acc2);
-      sumsq_f64(v[k].w, acc3);
+      sumsq_pair(v[k].x, acc[0], acc[1]);
+      sumsq_pair(v[k].y, acc[2], acc[3]);
+      sumsq_pair(v[k].z, acc[4], acc[5]);
+      sumsq_pair(v[k].w, acc[6], acc[7]);
     }
-    double ss = (acc0 + acc1) + (acc2 + acc3);
+    double ss = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     if (lane == 0) tail.partial[buf][warp] = ss;
@@ -247,44 +297,52 @@ __global__ void __launch_bounds__(kThreads) qk_norm_rope_kernel(const __grid_con
     const double rd = 1.0 / sqrt(((part[0] + part[1]) + (part[2] + part[3])) * p.inv_d + p.eps);
     const float r_hi = static_cast<float>(rd);
     const float r_lo = static_cast<float>(rd - static_cast<double>(r_hi));
-    const int pair0 = (u & 15) * 4;
-    const float4 cs0 = tail.rot[buf][pair0], cs1 = tail.rot[buf][pair0 + 1];
-    const float4 cs2 = tail.rot[buf][pair0 + 2], cs3 = tail.rot[buf][pair0 + 3];
-    const uint16_t* g = which ? p.gamma_k : p.gamma_q;
+    const uint64_t r2 = f2(r_hi, r_hi);
     uint16_t* x = p.qkv + tok * 3 * static_cast<int64_t>(p.D) + which * p.D;
+
+    // Pass A: y = bf16(x * g * r) for every pair held by this thread, with
+    // the exact rounding for the rare vectors near a rounding midpoint.
+    uint32_t y[VPT][4];
 #pragma unroll
     for (int k = 0; k < VPT; ++k) {
       const int vi = u + kRowThreads * k;
-      if (vi < p.nvec) {
-        const uint4 gv = ld_cached(g + 8 * vi);
-        const uint32_t xw[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
-        const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
-        uint32_t yw[4];
-        uint32_t near = 0xFFFFu;
+      // gammas: L1-resident, the same channels for every token
+      const uint4 gv = vi < p.nvec ? ld_cached(g + 8 * vi) : make_uint4(0, 0, 0, 0);
+      const uint32_t xw[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+      const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+      uint32_t near = 0xFFFFFFFFu;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) y[k][e] = norm_round(xw[e], gw[e], r2, near);
+      if ((near & 0xFFF8u) == 0u || (near & 0xFFF80000u) == 0u) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float xg0 = bf16_lo(xw[e]) * bf16_lo(gw[e]);  // exact: 8-bit x 8-bit significands
-          const float xg1 = bf16_hi(xw[e]) * bf16_hi(gw[e]);
-          const float v0 = xg0 * r_hi, v1 = xg1 * r_hi;
-          near = min(near, min(near_midpoint(v0), near_midpoint(v1)));
-          yw[e] = pack_bf16x2(v0, v1);
+          const uint32_t lo = round_exact(bf16_lo(xw[e]) * bf16_lo(gw[e]), r_hi, r_lo);
+          const uint32_t hi = round_exact(bf16_hi(xw[e]) * bf16_hi(gw[e]), r_hi, r_lo);
+          y[k][e] = lo | (hi << 16);
         }
-        if (near <= 4u) {
-          // Rare: some v_hi is within 2 ulps of a rounding midpoint.
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const uint32_t lo = round_exact(bf16_lo(xw[e]) * bf16_lo(gw[e]), r_hi, r_lo);
-            const uint32_t hi = round_exact(bf16_hi(xw[e]) * bf16_hi(gw[e]), r_hi, r_lo);
-            yw[e] = lo | (hi << 16);
-          }
-        }
-        uint4 o;
-        o.x = rotate_pair(yw[0], cs0);
-        o.y = rotate_pair(yw[1], cs1);
-        o.z = rotate_pair(yw[2], cs2);
-        o.w = rotate_pair(yw[3], cs3);
-        st_v4(x + 8 * vi, o);
       }
+    }
+    // Pass B: rotate, one pair position (4 per thread) at a time so that only
+    // its cos/sin operands are live.
+    const int pair0 = (u & 15) * 4;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float4 ra = tail.rot[rbuf][pair0 + e][0];
+      const float4 rb = tail.rot[rbuf][pair0 + e][1];
+#pragma unroll
+      for (int k = 0; k < VPT; ++k) y[k][e] = rotate(y[k][e], ra, rb);
+    }
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) {
+      const int vi = u + kRowThreads * k;
+      if (vi < p.nvec) st_v4(x + 8 * vi, make_uint4(y[k][0], y[k][1], y[k][2], y[k][3]));
+    }
+    rbuf = rnext;
+    s_next += step_mod;
+    if (s_next >= p.S) s_next -= p.S;
+    if (++stage == p.stages) {
+      stage = 0;
+      parity ^= 1u;
     }
   }
   if (tail.abort && tid == 0) {

@@ -78,9 +78,12 @@ struct NormRopeParams {
 struct alignas(16) NormSmemTail {
   uint64_t full[kMaxStages];
   double partial[2][8];            // per warp sums of squares, double-buffered by token parity
-  float4 rot[3][kPairs][2];        // per pair: (ch, sh, -sh, ch), (cl, sl, -sl, cl) -- cos/sin
-                                   // heads and tails as f32x2 operands; the table of
-                                   // iteration i+1 is written during iteration i
+  // Rotation operands of pair 4*g + e at [buf][e][g]: (ch, sh, -sh, ch) in
+  // rot_a, (cl, sl, -sl, cl) in rot_b -- cos/sin heads and tails as f32x2
+  // operands. A warp reads the 16 entries of one e: contiguous, no bank
+  // conflicts. The table of iteration i+1 is written during iteration i.
+  float4 rot_a[3][4][16];
+  float4 rot_b[3][4][16];
   int abort;
 };
 
@@ -129,7 +132,8 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
 
 // Rotation table entries of pair `pr` for sequence index s (one fp64 sincos):
 // cos/sin split into a 16-significant-bit head and a float tail.
-__device__ __forceinline__ void rotation(const NormRopeParams& p, int s, int pr, float4* dst) {
+__device__ __forceinline__ void rotation(const NormRopeParams& p, int s, int pr, float4& dst_a,
+                                         float4& dst_b) {
   const int q = s / p.W;  // frame * H + row
   const int pos = pr < kRowAxisPair0 ? q / p.H : (pr < kColAxisPair0 ? q - (q / p.H) * p.H : s - q * p.W);
   double sd, cd;
@@ -138,8 +142,8 @@ __device__ __forceinline__ void rotation(const NormRopeParams& p, int s, int pr,
   const float sh = __uint_as_float(__float_as_uint(static_cast<float>(sd)) & 0xFFFFFF00u);
   const float cl = static_cast<float>(cd - static_cast<double>(ch));
   const float sl = static_cast<float>(sd - static_cast<double>(sh));
-  dst[0] = make_float4(ch, sh, -sh, ch);
-  dst[1] = make_float4(cl, sl, -sl, cl);
+  dst_a = make_float4(ch, sh, -sh, ch);
+  dst_b = make_float4(cl, sl, -sl, cl);
 }
 
 // ---- packed fp32x2 arithmetic (one instruction for two lanes of a pair)
@@ -162,17 +166,31 @@ __device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
   return r;
 }
 
-// x^2 of both bf16 halves of w accumulated in fp64. A bf16 value's double
-// has the high word ((f32 bits >> 3) & 0x0FFFFFFF) + ((1023-127) << 20) and a
-// zero low word (the sign is dropped, irrelevant for a square; zero and
-// subnormal inputs map to ~2^-127, whose square is below 1e-76).
+// Exact products of the two bf16 halves of a and b (8-bit x 8-bit
+// significands fit a float): one mixed-precision FMA per half, no unpacking.
+__device__ __forceinline__ void prod_bf16x2(uint32_t a, uint32_t b, float& lo, float& hi) {
+  asm("{\n\t.reg .b16 al, ah, bl, bh;\n\t"
+      "mov.b32 {al, ah}, %2;\n\t"
+      "mov.b32 {bl, bh}, %3;\n\t"
+      "fma.rn.f32.bf16 %0, al, bl, 0f00000000;\n\t"
+      "fma.rn.f32.bf16 %1, ah, bh, 0f00000000;\n\t}"
+      : "=f"(lo), "=f"(hi)
+      : "r"(a), "r"(b));
+}
+
+// Exact fp64 value of a non-negative float with a 16-bit significand (a
+// square of a bf16): high word (bits >> 3) + ((1023-127) << 20), zero low
+// word. Zero and subnormal squares map to about 2^-127, negligible next to eps.
+__device__ __forceinline__ double square_to_f64(float sq) {
+  return __hiloint2double(static_cast<int>(__umulhi(__float_as_uint(sq), 1u << 29) + 0x38000000u), 0);
+}
+
+// x^2 of both bf16 halves of w accumulated in fp64.
 __device__ __forceinline__ void sumsq_pair(uint32_t w, double& acc_lo, double& acc_hi) {
-  const uint32_t hw_lo = (w & 0x7FFFu) * 8192u + 0x38000000u;
-  const uint32_t hw_hi = __umulhi(w & 0x7FFF0000u, 1u << 29) + 0x38000000u;
-  const double a = __hiloint2double(static_cast<int>(hw_lo), 0);
-  const double b = __hiloint2double(static_cast<int>(hw_hi), 0);
-  acc_lo = fma(a, a, acc_lo);
-  acc_hi = fma(b, b, acc_hi);
+  float s0, s1;
+  prod_bf16x2(w, w, s0, s1);
+  acc_lo += square_to_f64(s0);
+  acc_hi += square_to_f64(s1);
 }
 
 // One pair: v = x*g*r_hi (x*g is exact) rounded to bf16. `near` keeps the
@@ -180,9 +198,9 @@ __device__ __forceinline__ void sumsq_pair(uint32_t w, double& acc_lo, double& a
 // when v lies within a few fp32 ulps of a bf16 rounding midpoint (a carry
 // from the low lane only widens the high lane's window).
 __device__ __forceinline__ uint32_t norm_round(uint32_t xw, uint32_t gw, uint64_t r2, uint32_t& near) {
-  const uint64_t x = f2(bf16_lo(xw), bf16_hi(xw));
-  const uint64_t g = f2(bf16_lo(gw), bf16_hi(gw));
-  const uint64_t v = mul2(mul2(x, g), r2);
+  float xg0, xg1;
+  prod_bf16x2(xw, gw, xg0, xg1);
+  const uint64_t v = mul2(f2(xg0, xg1), r2);
   float v0, v1;
   f2_split(v, v0, v1);
   const uint32_t lows = __byte_perm(__float_as_uint(v0), __float_as_uint(v1), 0x5410);
@@ -240,7 +258,8 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const __grid_
   // incrementally (no 64-bit division in the loop).
   const int step_mod = static_cast<int>(step % p.S);
   int s_next = static_cast<int>(blockIdx.x % p.S);
-  if ((tid & 3) == 0) rotation(p, s_next, tid >> 2, tail.rot[0][tid >> 2]);
+  const int my_pr = tid >> 2;  // the pair whose rotation this thread computes (every 4th thread)
+  if ((tid & 3) == 0) rotation(p, s_next, my_pr, tail.rot_a[0][my_pr & 3][my_pr >> 2], tail.rot_b[0][my_pr & 3][my_pr >> 2]);
   s_next += step_mod;
   if (s_next >= p.S) s_next -= p.S;
   __syncthreads();
@@ -252,7 +271,10 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const __grid_
     const int buf = static_cast<int>(i & 1);
     // The next token's rotations, ahead of time (they do not depend on the data).
     const int rnext = rbuf == 2 ? 0 : rbuf + 1;
-    if ((tid & 3) == 0 && tok + step < p.tokens) rotation(p, s_next, tid >> 2, tail.rot[rnext][tid >> 2]);
+    if ((tid & 3) == 0 && tok + step < p.tokens) {
+      rotation(p, s_next, my_pr, tail.rot_a[rnext][my_pr & 3][my_pr >> 2],
+               tail.rot_b[rnext][my_pr & 3][my_pr >> 2]);
+    }
     if (!mbar_wait(smem_u32(&tail.full[stage]), parity, nullptr, kWaitLimitNs)) {
       tail.abort = 1;
       atomicOr(&g_norm_error_word, 1);
@@ -324,11 +346,10 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const __grid_
     }
     // Pass B: rotate, one pair position (4 per thread) at a time so that only
     // its cos/sin operands are live.
-    const int pair0 = (u & 15) * 4;
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const float4 ra = tail.rot[rbuf][pair0 + e][0];
-      const float4 rb = tail.rot[rbuf][pair0 + e][1];
+      const float4 ra = tail.rot_a[rbuf][e][u & 15];
+      const float4 rb = tail.rot_b[rbuf][e][u & 15];
 #pragma unroll
       for (int k = 0; k < VPT; ++k) y[k][e] = rotate(y[k][e], ra, rb);
     }

@@ -78,12 +78,12 @@ struct NormRopeParams {
 struct alignas(16) NormSmemTail {
   uint64_t full[kMaxStages];
   double partial[2][8];            // per warp sums of squares, double-buffered by token parity
-  // Rotation operands of pair 4*g + e at [buf][e][g]: (ch, sh, -sh, ch) in
-  // rot_a, (cl, sl, -sl, cl) in rot_b -- cos/sin heads and tails as f32x2
-  // operands. A warp reads the 16 entries of one e: contiguous, no bank
+  // Rotation operands, for two pairs a = 4g + 2h and b = a + 1 at once, as
+  // f32x2 lanes (a, b): rot[buf][h][0][g] = (ch, ch | sh, sh),
+  // [1] = (-sh, -sh | cl, cl), [2] = (sl, sl | -sl, -sl) -- cos/sin heads and
+  // tails. A warp reads the 16 entries of one (h, j): contiguous, no bank
   // conflicts. The table of iteration i+1 is written during iteration i.
-  float4 rot_a[3][4][16];
-  float4 rot_b[3][4][16];
+  float4 rot[3][2][3][16];
   int abort;
 };
 
@@ -130,10 +130,10 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
       : "memory");
 }
 
-// Rotation table entries of pair `pr` for sequence index s (one fp64 sincos):
-// cos/sin split into a 16-significant-bit head and a float tail.
-__device__ __forceinline__ void rotation(const NormRopeParams& p, int s, int pr, float4& dst_a,
-                                         float4& dst_b) {
+// Rotation operands of pair `pr` for sequence index s (one fp64 sincos):
+// cos/sin split into a 16-significant-bit head and a float tail, written into
+// its lane of the two-pair table entry.
+__device__ __forceinline__ void rotation(const NormRopeParams& p, int s, int pr, float4 (&t)[2][3][16]) {
   const int q = s / p.W;  // frame * H + row
   const int pos = pr < kRowAxisPair0 ? q / p.H : (pr < kColAxisPair0 ? q - (q / p.H) * p.H : s - q * p.W);
   double sd, cd;
@@ -142,8 +142,16 @@ __device__ __forceinline__ void rotation(const NormRopeParams& p, int s, int pr,
   const float sh = __uint_as_float(__float_as_uint(static_cast<float>(sd)) & 0xFFFFFF00u);
   const float cl = static_cast<float>(cd - static_cast<double>(ch));
   const float sl = static_cast<float>(sd - static_cast<double>(sh));
-  dst_a = make_float4(ch, sh, -sh, ch);
-  dst_b = make_float4(cl, sl, -sl, cl);
+  const int g = pr >> 2, h = (pr >> 1) & 1, side = pr & 1;
+  float* t0 = reinterpret_cast<float*>(&t[h][0][g]);
+  float* t1 = reinterpret_cast<float*>(&t[h][1][g]);
+  float* t2 = reinterpret_cast<float*>(&t[h][2][g]);
+  t0[side] = ch;
+  t0[2 + side] = sh;
+  t1[side] = -sh;
+  t1[2 + side] = cl;
+  t2[side] = sl;
+  t2[2 + side] = -sl;
 }
 
 // ---- packed fp32x2 arithmetic (one instruction for two lanes of a pair)
@@ -208,16 +216,28 @@ __device__ __forceinline__ uint32_t norm_round(uint32_t xw, uint32_t gw, uint64_
   return wan::sm100::pack_bf16x2(v0, v1);
 }
 
-__device__ __forceinline__ uint32_t rotate(uint32_t yw, const float4& A, const float4& B) {
-  const float y0 = bf16_lo(yw), y1 = bf16_hi(yw);
-  const uint64_t yy0 = f2(y0, y0), yy1 = f2(y1, y1);
-  // (y0 ch - y1 sh, y0 sh + y1 ch): head products are exact, one rounding.
-  uint64_t o = fma2(yy0, f2(A.x, A.y), mul2(yy1, f2(A.z, A.w)));
-  o = fma2(yy1, f2(B.z, B.w), o);  // + (-y1 sl, y1 cl)
-  o = fma2(yy0, f2(B.x, B.y), o);  // + (y0 cl, y0 sl)
-  float o0, o1;
+// Rotation of two adjacent pairs a = (y0, y1) in wa and b = (y2, y3) in wb,
+// lanes (a, b) of f32x2 operations: (y0 ch - y1 sh, y0 sh + y1 ch) per pair.
+// The head products (8-bit y x 16-bit head) are exact, so each head sum is
+// rounded once; the tails add their (2^-16 smaller) share.
+__device__ __forceinline__ void rotate2(uint32_t& wa, uint32_t& wb, const float4& t0, const float4& t1,
+                                        const float4& t2) {
+  const uint64_t ye = f2(bf16_lo(wa), bf16_lo(wb));  // (y0, y2)
+  const uint64_t yo = f2(bf16_hi(wa), bf16_hi(wb));  // (y1, y3)
+  const uint64_t ch = f2(t0.x, t0.y), sh = f2(t0.z, t0.w);
+  const uint64_t nsh = f2(t1.x, t1.y), cl = f2(t1.z, t1.w);
+  const uint64_t sl = f2(t2.x, t2.y), nsl = f2(t2.z, t2.w);
+  uint64_t e = fma2(ye, ch, mul2(yo, nsh));
+  e = fma2(yo, nsl, e);
+  e = fma2(ye, cl, e);
+  uint64_t o = fma2(ye, sh, mul2(yo, ch));
+  o = fma2(yo, cl, o);
+  o = fma2(ye, sl, o);
+  float e0, e1, o0, o1;
+  f2_split(e, e0, e1);
   f2_split(o, o0, o1);
-  return wan::sm100::pack_bf16x2(o0, o1);
+  wa = wan::sm100::pack_bf16x2(e0, o0);
+  wb = wan::sm100::pack_bf16x2(e1, o1);
 }
 
 template <int VPT>
@@ -259,7 +279,7 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const __grid_
   const int step_mod = static_cast<int>(step % p.S);
   int s_next = static_cast<int>(blockIdx.x % p.S);
   const int my_pr = tid >> 2;  // the pair whose rotation this thread computes (every 4th thread)
-  if ((tid & 3) == 0) rotation(p, s_next, my_pr, tail.rot_a[0][my_pr & 3][my_pr >> 2], tail.rot_b[0][my_pr & 3][my_pr >> 2]);
+  if ((tid & 3) == 0) rotation(p, s_next, my_pr, tail.rot[0]);
   s_next += step_mod;
   if (s_next >= p.S) s_next -= p.S;
   __syncthreads();
@@ -271,10 +291,7 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const __grid_
     const int buf = static_cast<int>(i & 1);
     // The next token's rotations, ahead of time (they do not depend on the data).
     const int rnext = rbuf == 2 ? 0 : rbuf + 1;
-    if ((tid & 3) == 0 && tok + step < p.tokens) {
-      rotation(p, s_next, my_pr, tail.rot_a[rnext][my_pr & 3][my_pr >> 2],
-               tail.rot_b[rnext][my_pr & 3][my_pr >> 2]);
-    }
+    if ((tid & 3) == 0 && tok + step < p.tokens) rotation(p, s_next, my_pr, tail.rot[rnext]);
     if (!mbar_wait(smem_u32(&tail.full[stage]), parity, nullptr, kWaitLimitNs)) {
       tail.abort = 1;
       atomicOr(&g_norm_error_word, 1);
@@ -344,14 +361,15 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const __grid_
         }
       }
     }
-    // Pass B: rotate, one pair position (4 per thread) at a time so that only
-    // its cos/sin operands are live.
+    // Pass B: rotate, two pair positions (of the 4 per thread) at a time so
+    // that only their cos/sin operands are live.
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float4 ra = tail.rot_a[rbuf][e][u & 15];
-      const float4 rb = tail.rot_b[rbuf][e][u & 15];
+    for (int h = 0; h < 2; ++h) {
+      const float4 t0 = tail.rot[rbuf][h][0][u & 15];
+      const float4 t1 = tail.rot[rbuf][h][1][u & 15];
+      const float4 t2 = tail.rot[rbuf][h][2][u & 15];
 #pragma unroll
-      for (int k = 0; k < VPT; ++k) y[k][e] = rotate(y[k][e], ra, rb);
+      for (int k = 0; k < VPT; ++k) rotate2(y[k][2 * h], y[k][2 * h + 1], t0, t1, t2);
     }
 #pragma unroll
     for (int k = 0; k < VPT; ++k) {

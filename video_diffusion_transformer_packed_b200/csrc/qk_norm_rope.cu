@@ -51,7 +51,7 @@ constexpr int kPairs = kHeadDim / 2;
 constexpr int kThreads = 256;    // warps 0-3: the Q row of a token, warps 4-7: its K row
 constexpr int kRowThreads = 128;
 constexpr int kMaxStages = 8;
-constexpr uint32_t kStageBudget = 72 * 1024;  // ring bytes per CTA (3 CTAs fit an SM)
+constexpr uint32_t kStageBudget = 48 * 1024;  // ring bytes per CTA
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 // Pair index where the row axis and the column axis start (split 44/42/42).
 constexpr int kRowAxisPair0 = 44 / 2;

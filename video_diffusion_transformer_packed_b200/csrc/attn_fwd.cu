@@ -74,6 +74,18 @@ constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 2 + 1;  // q, kv full/empty, 
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + alignment slack
 
+// 2^x on the FMA pipe for part of the probabilities (the rest use MUFU ex2):
+// x = n + f, n = round(x) by the 1.5*2^23 magic add, f in [-1/2, 1/2],
+// 2^x = 2^n * p(f) with p the degree-3 minimax fit of 2^f in relative error
+// (max 7.5e-5) produced by exp2_poly.py next to this file; 2^n is applied by
+// adding n to the exponent field.
+constexpr uint32_t kPolyC0 = 0x3F7FFB49u, kPolyC1 = 0x3F31798Du, kPolyC2 = 0x3E786F0Du,
+                   kPolyC3 = 0x3D61FBB0u;
+constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+// Pairs of score columns whose exponentials go to the FMA pipe: 3 of every 8
+// (the MUFU unit alone needs as long as the tensor core for one tile).
+__host__ __device__ constexpr bool poly_pair(int e) { return (e & 7) == 2 || (e & 7) == 5 || (e & 7) == 7; }
+
 // Error-word site codes.
 constexpr int kErrProducer = 1, kErrMma = 2, kErrSoftmax = 4, kErrEpilogue = 8, kErrDrain = 16;
 
@@ -236,6 +248,28 @@ __device__ void run_mma(const AttnParams& p, uint32_t smem, Bars bars, volatile 
   if (!mbar_wait(bars.drain(), 0, nullptr, kWaitLimitNs)) atomicOr(&g_attn_error_word, kErrDrain);
 }
 
+// 2^x for both lanes of a packed pair on the FMA pipe (x clamped to >= -126,
+// below which the result is under 2^-126 and only its smallness matters).
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
+  float x0, x1;
+  f2_split(x2, x0, x1);
+  x2 = f2(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+  const uint64_t magic = f2(kMagic, kMagic);
+  const uint64_t j = add2(x2, magic);        // round(x) in the low mantissa bits
+  const uint64_t f = sub2(x2, sub2(j, magic));  // x - round(x), in [-1/2, 1/2]
+  uint64_t p = fma2(f2(__uint_as_float(kPolyC3), __uint_as_float(kPolyC3)), f,
+                    f2(__uint_as_float(kPolyC2), __uint_as_float(kPolyC2)));
+  p = fma2(p, f, f2(__uint_as_float(kPolyC1), __uint_as_float(kPolyC1)));
+  p = fma2(p, f, f2(__uint_as_float(kPolyC0), __uint_as_float(kPolyC0)));
+  float p0, p1, j0, j1;
+  f2_split(p, p0, p1);
+  f2_split(j, j0, j1);
+  // the magic's own bits vanish when shifted by 23 (its lowest set bit is 2^22)
+  const float r0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(j0) << 23));
+  const float r1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(j1) << 23));
+  return f2(r0, r1);
+}
+
 // ----------------------------------------------------------------- softmax
 __device__ void run_softmax(const AttnParams& p, Bars bars, volatile int* abort, uint32_t tmem,
                             int t, int quarter, int lane, int b, int h, int qp) {
@@ -264,7 +298,8 @@ __device__ void run_softmax(const AttnParams& p, Bars bars, volatile int* abort,
     }
     float mx = __uint_as_float(sr[0]);
 #pragma unroll
-    for (int c = 1; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(sr[c]));
+    for (int c = 1; c < 127; c += 2) mx = max3(mx, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+    mx = fmaxf(mx, __uint_as_float(sr[127]));
     const float m_cand = mx * sl2;
     const bool raise = m_cand > m_run + kRescaleThreshold;
     float alpha = 1.f;
@@ -287,20 +322,35 @@ __device__ void run_softmax(const AttnParams& p, Bars bars, volatile int* abort,
       }
       tmem_wait_st();
     }
-    const float neg_m = -m_run;
-    float sum = 0.f;
+    // p = 2^(s * scale * log2(e) - m), two columns per packed instruction.
+    const uint64_t sl2_2 = f2(sl2, sl2);
+    const uint64_t negm2 = f2(-m_run, -m_run);
+    uint64_t sum2 = f2(0.f, 0.f);
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
       uint32_t pk[32];
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
-        const float p0 = ex2(fmaf(__uint_as_float(sr[64 * half + 2 * e]), sl2, neg_m));
-        const float p1 = ex2(fmaf(__uint_as_float(sr[64 * half + 2 * e + 1]), sl2, neg_m));
-        sum += p0 + p1;
+        const int pe = 32 * half + e;  // pair index: columns 2pe, 2pe+1
+        const uint64_t x2 = fma2(f2(__uint_as_float(sr[2 * pe]), __uint_as_float(sr[2 * pe + 1])), sl2_2, negm2);
+        uint64_t p2;
+        if (poly_pair(pe)) {
+          p2 = exp2_poly2(x2);
+        } else {
+          float x0, x1;
+          f2_split(x2, x0, x1);
+          p2 = f2(ex2(x0), ex2(x1));
+        }
+        sum2 = add2(sum2, p2);
+        float p0, p1;
+        f2_split(p2, p0, p1);
         pk[e] = pack_bf16x2(p0, p1);
       }
       tmem_st32(tS + 32 * half, pk);
     }
+    float sum_lo, sum_hi;
+    f2_split(sum2, sum_lo, sum_hi);
+    const float sum = sum_lo + sum_hi;
     tmem_wait_st();
     tc_fence_before();
     mbar_arrive(bars.p_full(t));

@@ -46,6 +46,11 @@
 namespace wan {
 namespace {
 
+using wan::sm100::f2;
+using wan::sm100::f2_split;
+using wan::sm100::fma2;
+using wan::sm100::mul2;
+
 constexpr int kHeadDim = 128;
 constexpr int kPairs = kHeadDim / 2;
 constexpr int kThreads = 256;    // warps 0-3: the Q row of a token, warps 4-7: its K row
@@ -152,26 +157,6 @@ __device__ __forceinline__ void rotation(const NormRopeParams& p, int s, int pr,
   t1[2 + side] = cl;
   t2[side] = sl;
   t2[2 + side] = -sl;
-}
-
-// ---- packed fp32x2 arithmetic (one instruction for two lanes of a pair)
-__device__ __forceinline__ uint64_t f2(float lo, float hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1,%2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ void f2_split(uint64_t v, float& lo, float& hi) {
-  asm("mov.b64 {%0,%1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t r;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-  return r;
 }
 
 // Exact products of the two bf16 halves of a and b (8-bit x 8-bit

@@ -6,7 +6,7 @@
 #include <cstdint>
 #include <mutex>
 
-#include "../../include/wan_attn.h"
+#include "wan_attn.h"  // include/ is on the include path
 #include "wan_kernels.h"
 
 namespace {

@@ -9,35 +9,25 @@
 // the packed [Q | K | V] allocation with no repack (TensorRT-LLM PR
 // "[visual_gen] Optimize Wan2.2 Dataflow", "Packed QKV Profiling Details").
 //
-// Design. A cluster of two CTAs (a CTA pair, one per SM) owns 512 query rows
-// of one (batch, head): CTA v holds query tiles t = 0, 1 of 128 rows each,
-// rows 512*qq + 256*t + 128*v. The tensor-core work runs as CTA-pair MMAs
-// (tcgen05 cta_group::2, M = 256): the even CTA's MMA thread issues every
-// MMA for both CTAs; each CTA supplies its own 128 rows of the A operand and
-// HALF of the B operand -- 64 of the 128 keys of a K tile, 64 of the 128 head
-// dims of a V tile -- which halves the shared-memory operand and TMA traffic
-// per SM compared with single-CTA 128 x 128 MMAs (those left the tensor pipe
-// waiting on shared-memory operand reads).
-//   warp 8      TMA producer (both CTAs): Q tiles once, then the K_j / V_j
-//               halves into an 8-slot ring of 16 KB; completion counted on the
-//               even CTA's barriers (3D tensor map over [B][S][3D]; rows past
-//               S read as zeros within the batch). No multicast.
-//   warp 9      MMA issuer (even CTA): S_t = Q_t K_j^T into TMEM, then
-//               O_t += P_t V_j with P_t read from TMEM; the two query tiles
-//               ping-pong so one tile's softmax overlaps the other's MMAs.
-//               Commits are multicast to both CTAs' barriers.
-//   warps 0-3   softmax of tile 0, warps 4-7 of tile 1 (both CTAs): thread r
-//               owns query row r (TMEM lane r); online softmax in base 2 with
-//               the running max raised (and O rescaled in TMEM) only when a
-//               tile's max exceeds it by more than 2^8 -- exact after the final
-//               division. P is rounded to bf16 and written over S in TMEM;
-//               readiness is signalled to the even CTA's barrier.
-// TMEM columns (each CTA): S_0 [0,128), S_1 [128,256), O_0 [256,384), O_1 [384,512).
+// Design (one CTA = one (batch, head) and two 128-row query tiles):
+//   warp 8      TMA producer: Q tiles once, then K_j / V_j tiles into a
+//               4-slot shared-memory ring (128-byte swizzle, 3D tensor map
+//               over [B][S][3D] so that rows past S read as zeros per batch).
+//   warp 9      MMA issuer (one thread): tcgen05.mma S_t = Q_t K_j^T into
+//               TMEM, then O_t += P_t V_j with P_t read from TMEM. The two
+//               query tiles ping-pong: while one tile's softmax runs, the
+//               tensor core works on the other tile.
+//   warps 0-3   softmax of tile 0, warps 4-7 softmax of tile 1: thread r owns
+//               query row r (TMEM lane r). Online softmax in base 2; the
+//               running max is only raised (and O rescaled in TMEM) when a
+//               tile's max exceeds it by more than 2^8, which keeps the
+//               result exact after the final division while skipping almost
+//               all rescales. P is rounded to bf16 and written over S in TMEM.
+// TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,384), O_1 [384,512).
 //
 // Every mbarrier wait is bounded (wall-clock limit); a wait that gives up
-// sets a block-wide abort flag and a device error word; the block then drains
-// what it started, meets its partner at the final cluster barrier, frees TMEM
-// and exits.
+// sets a block-wide abort flag and a device error word, and the block then
+// drains its own copies and MMAs, frees TMEM and exits.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -55,14 +45,12 @@ namespace {
 
 using namespace wan::sm100;
 
-constexpr int kBM = 128;  // query rows per tile (per CTA)
-constexpr int kBN = 128;  // keys per iteration
+constexpr int kBM = 128;  // query rows per tile
+constexpr int kBN = 128;  // keys per tile
 constexpr int kHD = 128;  // head dim
-constexpr int kPairRows = 4 * kBM;  // query rows per CTA pair
-constexpr int kStages = 8;          // ring slots, each one K half or one V half
-constexpr int kTileBytes = kBM * kHD * 2;  // 32 KB: one 128 x 128 bf16 Q tile
-constexpr int kBoxBytes = 64 * 64 * 2;     // 8 KB: one TMA box of 64 rows x 64 columns
-constexpr int kSlotBytes = 2 * kBoxBytes;  // 16 KB: a K half (64 keys x 128) or V half (128 keys x 64)
+constexpr int kStages = 4;
+constexpr int kTileBytes = kBM * kHD * 2;  // 32 KB: one 128 x 128 bf16 tile
+constexpr int kBoxBytes = kTileBytes / 2;  // 16 KB: 128 rows x 64 columns (one TMA box)
 constexpr int kThreads = 384;  // 3 warpgroups: softmax tile 0, softmax tile 1, load/MMA
 constexpr int kLoadWarp = 8;
 constexpr int kMmaWarp = 9;
@@ -77,32 +65,17 @@ static_assert(128 * kCtlRegs + 256 * kSoftmaxRegs <= kThreads * kLaunchRegs, "re
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
 constexpr float kRescaleThreshold = 8.0f;         // log2 of the largest tolerated growth
-constexpr uint16_t kBothCtas = 0x3;
 
-// Shared memory map (offsets from a 1024-byte aligned base; identical in
-// both CTAs of a pair, which the CTA-pair MMAs rely on).
+// Shared memory map (offsets from a 1024-byte aligned base).
 constexpr int kOffQ = 0;                              // 2 tiles
-constexpr int kOffKV = kOffQ + 2 * kTileBytes;        // kStages slots
-constexpr int kOffBar = kOffKV + kStages * kSlotBytes;
+constexpr int kOffKV = kOffQ + 2 * kTileBytes;        // kStages tiles
+constexpr int kOffBar = kOffKV + kStages * kTileBytes;
 constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 2 + 1;  // q, kv full/empty, s, p, o, drain
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + alignment slack
 
-// 2^x on the FMA pipe for part of the probabilities (the rest use MUFU ex2):
-// x = n + f, n = round(x) by the 1.5*2^23 magic add, f in [-1/2, 1/2],
-// 2^x = 2^n * p(f) with p the degree-3 minimax fit of 2^f in relative error
-// (max 7.5e-5) produced by exp2_poly.py next to this file; 2^n is applied by
-// adding n to the exponent field.
-constexpr uint32_t kPolyC0 = 0x3F7FFB49u, kPolyC1 = 0x3F31798Du, kPolyC2 = 0x3E786F0Du,
-                   kPolyC3 = 0x3D61FBB0u;
-constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
-// Pairs of score columns whose exponentials go to the FMA pipe: 3 of every 8
-// (the MUFU unit alone needs as long as the tensor core for one tile).
-__host__ __device__ constexpr bool poly_pair(int e) { return (e & 7) == 2 || (e & 7) == 5 || (e & 7) == 7; }
-
 // Error-word site codes.
-constexpr int kErrProducer = 1, kErrMma = 2, kErrSoftmax = 4, kErrEpilogue = 8, kErrDrain = 16,
-              kErrTmem = 32;
+constexpr int kErrProducer = 1, kErrMma = 2, kErrSoftmax = 4, kErrEpilogue = 8, kErrDrain = 16;
 
 __device__ int g_attn_error_word;
 
@@ -111,15 +84,12 @@ struct AttnParams {
   int32_t S;
   int32_t heads;
   int32_t D;
-  int32_t q_quads;  // ceil(S / 512): CTA pairs per (batch, head)
+  int32_t q_pairs;  // ceil(S / 256): CTAs per (batch, head)
   int32_t n_kv;     // ceil(S / 128)
   float scale_log2; // scale * log2(e)
 };
 
 // Barrier addresses (32-bit shared-memory addresses, 8 bytes apart).
-//  q_full, kv_full, p_full, drain: used in the even CTA (both CTAs' loads and
-//    softmax threads arrive there);
-//  kv_empty, s_full, o_full: in each CTA (the MMA commits are multicast).
 struct Bars {
   uint32_t base;
   __device__ __forceinline__ uint32_t q_full() const { return base; }
@@ -138,24 +108,15 @@ __device__ __forceinline__ void flag_error(volatile int* abort, int site) {
 }
 
 // ---------------------------------------------------------------- producer
-// Both CTAs: this CTA's Q tiles, then its halves of K_j (keys 64v..64v+63 of
-// the tile) and V_j (head dims 64v..64v+63), completion on the even CTA's
-// barriers. The even CTA also announces the byte counts of both CTAs.
 __device__ void run_producer(const CUtensorMap* tmap, const AttnParams& p, uint32_t smem,
-                             Bars bars, uint32_t rank, volatile int* abort, int* issued, int b,
-                             int h, int qq) {
+                             Bars bars, volatile int* abort, int* issued, int b, int h, int qp) {
   grid_dependency_wait();  // the packed buffer may still be written by the norm kernel
-  const bool leader = rank == 0;
-  const int xq = h * kHD, xk = p.D + h * kHD, xv = 2 * p.D + h * kHD + 64 * static_cast<int>(rank);
-  const uint32_t q_bar = map_to_cta(bars.q_full(), 0);
-  if (leader) mbar_arrive_expect_tx(bars.q_full(), 2 * 2 * kTileBytes);  // both CTAs' Q tiles
+  const int xq = h * kHD, xk = p.D + h * kHD, xv = 2 * p.D + h * kHD;
+  mbar_arrive_expect_tx(bars.q_full(), 2 * kTileBytes);
   for (int t = 0; t < 2; ++t) {
-    const int row0 = kPairRows * qq + 2 * kBM * t + kBM * static_cast<int>(rank);
-    for (int half = 0; half < 2; ++half) {       // head dims 0-63, 64-127
-      for (int rh = 0; rh < 2; ++rh) {           // rows 0-63, 64-127
-        tma_load_3d_pair(smem + kOffQ + t * kTileBytes + half * (kTileBytes / 2) + rh * kBoxBytes, tmap, q_bar,
-                         xq + 64 * half, row0 + 64 * rh, b);
-      }
+    for (int half = 0; half < 2; ++half) {
+      tma_load_3d(smem + kOffQ + t * kTileBytes + half * kBoxBytes, tmap, bars.q_full(),
+                  xq + 64 * half, (2 * qp + t) * kBM, b);
     }
   }
   bool ok = true;
@@ -168,154 +129,119 @@ __device__ void run_producer(const CUtensorMap* tmap, const AttnParams& p, uint3
       ok = false;
       break;
     }
-    if (leader) mbar_arrive_expect_tx(bars.kv_full(slot), 2 * kSlotBytes);  // both halves
-    const uint32_t bar = map_to_cta(bars.kv_full(slot), 0);
-    const uint32_t dst = smem + kOffKV + slot * kSlotBytes;
-    const int key0 = (i >> 1) * kBN;
-    if ((i & 1) == 0) {
-      // K half: keys key0 + 64*rank .. +63, all 128 head dims (two column boxes)
-      const int y = key0 + 64 * static_cast<int>(rank);
-      tma_load_3d_pair(dst, tmap, bar, xk, y, b);
-      tma_load_3d_pair(dst + kBoxBytes, tmap, bar, xk + 64, y, b);
-    } else {
-      // V half: all 128 keys (two row boxes), head dims 64*rank .. +63
-      tma_load_3d_pair(dst, tmap, bar, xv, key0, b);
-      tma_load_3d_pair(dst + kBoxBytes, tmap, bar, xv, key0 + 64, b);
-    }
+    mbar_arrive_expect_tx(bars.kv_full(slot), kTileBytes);
+    const int x = (i & 1) ? xv : xk;
+    const int y = (i >> 1) * kBN;
+    const uint32_t dst = smem + kOffKV + slot * kTileBytes;
+    tma_load_3d(dst, tmap, bars.kv_full(slot), x, y, b);
+    tma_load_3d(dst + kBoxBytes, tmap, bars.kv_full(slot), x + 64, y, b);
     issued[slot] = use + 1;
   }
   if (!ok) flag_error(abort, kErrProducer);
 }
 
-// After an abort, the even CTA waits (bounded, ignoring the abort flag) for
-// every load phase it announced, so no bulk copy lands after the pair exits.
+// After an abort, waits (bounded, ignoring the abort flag) for every copy the
+// producer started, so that no bulk copy lands after the block has exited.
 __device__ void drain_producer(Bars bars, const int* issued) {
   for (int s = 0; s < kStages; ++s) {
-    if (issued[s] > 0 && !mbar_wait_cluster(bars.kv_full(s), (issued[s] - 1) & 1, nullptr, kWaitLimitNs)) {
+    if (issued[s] > 0 && !mbar_wait(bars.kv_full(s), (issued[s] - 1) & 1, nullptr, kWaitLimitNs)) {
       atomicOr(&g_attn_error_word, kErrDrain);
     }
   }
-  if (!mbar_wait_cluster(bars.q_full(), 0, nullptr, kWaitLimitNs)) atomicOr(&g_attn_error_word, kErrDrain);
+  if (!mbar_wait(bars.q_full(), 0, nullptr, kWaitLimitNs)) atomicOr(&g_attn_error_word, kErrDrain);
 }
 
 // -------------------------------------------------------------- MMA issuer
-// Even CTA only. Descriptors name this CTA's shared memory; the partner's
-// halves sit at the same offsets in its own shared memory.
 __device__ void run_mma(const AttnParams& p, uint32_t smem, Bars bars, volatile int* abort,
                         uint32_t tmem) {
-  constexpr uint32_t kIdescQK = idesc_bf16_f32(2 * kBM, kBN, 0);  // M = 256 over the pair
-  constexpr uint32_t kIdescPV = idesc_bf16_f32(2 * kBM, kHD, 1);
+  constexpr uint32_t kIdescQK = idesc_bf16_f32(kBM, kBN, 0);
+  constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, kHD, 1);
   // Descriptors are built once; a step only adds a byte offset (in 16-byte
   // units) to the start-address field, which cannot carry out of its 14 bits
   // because shared-memory addresses stay below 2^18.
   //
-  // S_t = Q_t K^T, K = 128 head dims in 8 steps of 16. Q_t: 128 rows, two
-  // 64-column halves 16 KB apart; K half: 64 keys, two 64-column halves 8 KB
-  // apart. Both 128-byte swizzled, 8-row groups 1024 bytes apart; a 16-element
-  // step inside a half advances the start address by 32 bytes.
+  // S_t = Q_t K^T: K = 128 head dims in 8 steps of 16; each 64-dim half of a
+  // tile is one 128-byte-swizzled box, and a 16-element step inside a box
+  // advances the start address by 32 bytes.
   const uint64_t q_desc0 = smem_desc_sw128(smem + kOffQ, 16, 1024);
   const uint64_t k_desc0 = smem_desc_sw128(smem + kOffKV, 16, 1024);
-  // V half [key][64 dims] is an N-major B: 8-key groups 1024 bytes apart; a
-  // 16-key step advances 2048 bytes; the 64 dims fill one swizzle span.
-  const uint64_t v_desc0 = smem_desc_sw128(smem + kOffKV, kSlotBytes, 1024);
+  // V [key][dim] is an N-major B: 8-key groups 1024 bytes apart, the two
+  // 64-dim halves one box (16 KB) apart; a 16-key step advances 2048 bytes.
+  const uint64_t v_desc0 = smem_desc_sw128(smem + kOffKV, kBoxBytes, 1024);
 
   auto issue_qk = [&](int t, int slot) {
     const uint32_t a0 = (t * kTileBytes) >> 4;
-    const uint32_t b0 = (slot * kSlotBytes) >> 4;
+    const uint32_t b0 = (slot * kTileBytes) >> 4;
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
-      const uint32_t aoff = ((kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32) >> 4;
-      const uint32_t boff = ((kk >> 2) * kBoxBytes + (kk & 3) * 32) >> 4;
-      mma_ss_pair(tmem + t * 128, desc_add(q_desc0, a0 + aoff), desc_add(k_desc0, b0 + boff), kIdescQK,
-                  kk > 0 ? 1u : 0u);
+      const uint32_t off = ((kk >> 2) * kBoxBytes + (kk & 3) * 32) >> 4;
+      mma_ss(tmem + t * 128, desc_add(q_desc0, a0 + off), desc_add(k_desc0, b0 + off), kIdescQK,
+             kk > 0 ? 1u : 0u);
     }
   };
   // O_t += P_t V: P_t (bf16, 64 TMEM columns over S_t) is the A operand.
   auto issue_pv = [&](int t, int slot, uint32_t acc) {
-    const uint32_t b0 = (slot * kSlotBytes) >> 4;
+    const uint32_t b0 = (slot * kTileBytes) >> 4;
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
-      mma_ts_pair(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, desc_add(v_desc0, b0 + kk * (2048 >> 4)),
-                  kIdescPV, kk > 0 ? 1u : acc);
+      mma_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, desc_add(v_desc0, b0 + kk * (2048 >> 4)),
+             kIdescPV, kk > 0 ? 1u : acc);
     }
   };
   auto wait_item = [&](int i) -> bool {
-    return mbar_wait_cluster(bars.kv_full(i % kStages), (i / kStages) & 1, abort, kWaitLimitNs);
+    return mbar_wait(bars.kv_full(i % kStages), (i / kStages) & 1, abort, kWaitLimitNs);
   };
 
-  bool ok = mbar_wait_cluster(bars.q_full(), 0, abort, kWaitLimitNs) && wait_item(0);
+  bool ok = mbar_wait(bars.q_full(), 0, abort, kWaitLimitNs) && wait_item(0);
   if (ok) {
     tc_fence_after();
     issue_qk(0, 0);
-    mma_commit_pair(bars.s_full(0), kBothCtas);
+    mma_commit(bars.s_full(0));
     issue_qk(1, 0);
-    mma_commit_pair(bars.s_full(1), kBothCtas);
-    mma_commit_pair(bars.kv_empty(0), kBothCtas);
+    mma_commit(bars.s_full(1));
+    mma_commit(bars.kv_empty(0));
   }
 #pragma unroll 1
   for (int j = 0; j < p.n_kv && ok; ++j) {
     const int iv = 2 * j + 1, ik = 2 * j + 2;
     const bool more = j + 1 < p.n_kv;
     const uint32_t acc = j > 0 ? 1u : 0u;
-    if (!wait_item(iv) || !mbar_wait_cluster(bars.p_full(0), j & 1, abort, kWaitLimitNs)) { ok = false; break; }
+    if (!wait_item(iv) || !mbar_wait(bars.p_full(0), j & 1, abort, kWaitLimitNs)) { ok = false; break; }
     tc_fence_after();
     issue_pv(0, iv % kStages, acc);
     if (more) {
       if (!wait_item(ik)) { ok = false; break; }
       tc_fence_after();
       issue_qk(0, ik % kStages);
-      mma_commit_pair(bars.s_full(0), kBothCtas);
+      mma_commit(bars.s_full(0));
     }
-    if (!mbar_wait_cluster(bars.p_full(1), j & 1, abort, kWaitLimitNs)) { ok = false; break; }
+    if (!mbar_wait(bars.p_full(1), j & 1, abort, kWaitLimitNs)) { ok = false; break; }
     tc_fence_after();
     issue_pv(1, iv % kStages, acc);
-    mma_commit_pair(bars.kv_empty(iv % kStages), kBothCtas);
+    mma_commit(bars.kv_empty(iv % kStages));
     if (more) {
       issue_qk(1, ik % kStages);
-      mma_commit_pair(bars.s_full(1), kBothCtas);
-      mma_commit_pair(bars.kv_empty(ik % kStages), kBothCtas);
+      mma_commit(bars.s_full(1));
+      mma_commit(bars.kv_empty(ik % kStages));
     }
   }
   if (ok) {
-    mma_commit_pair(bars.o_full(0), kBothCtas);
-    mma_commit_pair(bars.o_full(1), kBothCtas);
+    mma_commit(bars.o_full(0));
+    mma_commit(bars.o_full(1));
   } else {
     flag_error(abort, kErrMma);
   }
-  // Every MMA this thread issued completes before either CTA releases TMEM.
-  mma_commit_pair(bars.drain(), 0x1);
+  // Every MMA this thread issued completes before TMEM can be released.
+  mma_commit(bars.drain());
   if (!mbar_wait(bars.drain(), 0, nullptr, kWaitLimitNs)) atomicOr(&g_attn_error_word, kErrDrain);
-}
-
-// 2^x for both lanes of a packed pair on the FMA pipe (x clamped to >= -126,
-// below which the result is under 2^-126 and only its smallness matters).
-__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
-  float x0, x1;
-  f2_split(x2, x0, x1);
-  x2 = f2(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
-  const uint64_t magic = f2(kMagic, kMagic);
-  const uint64_t j = add2(x2, magic);        // round(x) in the low mantissa bits
-  const uint64_t f = sub2(x2, sub2(j, magic));  // x - round(x), in [-1/2, 1/2]
-  uint64_t p = fma2(f2(__uint_as_float(kPolyC3), __uint_as_float(kPolyC3)), f,
-                    f2(__uint_as_float(kPolyC2), __uint_as_float(kPolyC2)));
-  p = fma2(p, f, f2(__uint_as_float(kPolyC1), __uint_as_float(kPolyC1)));
-  p = fma2(p, f, f2(__uint_as_float(kPolyC0), __uint_as_float(kPolyC0)));
-  float p0, p1, j0, j1;
-  f2_split(p, p0, p1);
-  f2_split(j, j0, j1);
-  // the magic's own bits vanish when shifted by 23 (its lowest set bit is 2^22)
-  const float r0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(j0) << 23));
-  const float r1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(j1) << 23));
-  return f2(r0, r1);
 }
 
 // ----------------------------------------------------------------- softmax
 __device__ void run_softmax(const AttnParams& p, Bars bars, volatile int* abort, uint32_t tmem,
-                            uint32_t rank, int t, int quarter, int lane, int b, int h, int qq) {
+                            int t, int quarter, int lane, int b, int h, int qp) {
   const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
   const uint32_t tS = tmem + lane_base + t * 128;
   const uint32_t tO = tmem + lane_base + 256 + t * 128;
-  const uint32_t p_bar = map_to_cta(bars.p_full(t), 0);  // the even CTA's barrier
   const float sl2 = p.scale_log2;
   float m_run = -INFINITY;  // running max, already in scaled log2 units
   float l_run = 0.f;
@@ -381,17 +307,10 @@ __device__ void run_softmax(const AttnParams& p, Bars bars, volatile int* abort,
       for (int e = 0; e < 32; ++e) {
         const int pe = 32 * half + e;  // pair index: columns 2pe, 2pe+1
         const uint64_t x2 = fma2(f2(__uint_as_float(sr[2 * pe]), __uint_as_float(sr[2 * pe + 1])), sl2_2, negm2);
-        uint64_t p2;
-        if (poly_pair(pe)) {
-          p2 = exp2_poly2(x2);
-        } else {
-          float x0, x1;
-          f2_split(x2, x0, x1);
-          p2 = f2(ex2(x0), ex2(x1));
-        }
-        sum2[e & 3] = add2(sum2[e & 3], p2);
-        float p0, p1;
-        f2_split(p2, p0, p1);
+        float x0, x1;
+        f2_split(x2, x0, x1);
+        const float p0 = ex2(x0), p1 = ex2(x1);
+        sum2[e & 3] = add2(sum2[e & 3], f2(p0, p1));
         pk[e] = pack_bf16x2(p0, p1);
       }
       tmem_st32(tS + 32 * half, pk);
@@ -401,7 +320,7 @@ __device__ void run_softmax(const AttnParams& p, Bars bars, volatile int* abort,
     const float sum = sum_lo + sum_hi;
     tmem_wait_st();
     tc_fence_before();
-    mbar_arrive_cluster(p_bar);
+    mbar_arrive(bars.p_full(t));
     l_run += sum;
   }
   if (!ok) {
@@ -414,7 +333,7 @@ __device__ void run_softmax(const AttnParams& p, Bars bars, volatile int* abort,
   }
   tc_fence_after();
   const float inv_l = 1.f / l_run;
-  const int row = kPairRows * qq + 2 * kBM * t + kBM * static_cast<int>(rank) + quarter * 32 + lane;
+  const int row = (2 * qp + t) * kBM + quarter * 32 + lane;
   uint16_t* dst = p.out + (static_cast<int64_t>(b) * p.S + row) * p.D + h * kHD;
 #pragma unroll 1
   for (int c = 0; c < 4; ++c) {
@@ -446,10 +365,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_ctarank();  // 0: the even CTA, which issues the MMAs
-  const int pair = blockIdx.x >> 1;
-  const int qq = pair % p.q_quads;
-  const int bh = pair / p.q_quads;
+  const int qp = blockIdx.x % p.q_pairs;
+  const int bh = blockIdx.x / p.q_pairs;
   const int b = bh / p.heads;
   const int h = bh % p.heads;
 
@@ -461,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(bars.s_full(t), 1);
-      mbar_init(bars.p_full(t), 2 * 128);  // softmax threads of both CTAs
+      mbar_init(bars.p_full(t), 128);
       mbar_init(bars.o_full(t), 1);
     }
     mbar_init(bars.drain(), 1);
@@ -470,41 +387,34 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
   }
   if (warp == kMmaWarp) {
-    tmem_alloc_pair(tmem_holder, kTmemCols);
-    tmem_relinquish_pair();
+    tmem_alloc(tmem_holder, kTmemCols);
+    tmem_relinquish();
   }
   if (warp == kLoadWarp && lane == 0) tma_prefetch_desc(&tmap);
   tc_fence_before();
-  cluster_sync();  // both CTAs' barriers initialised and TMEM allocated
+  __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  // The pair's MMAs address both CTAs' TMEM at the even CTA's column base.
-  if (rank == 1 && threadIdx.x == 0 && ld_shared_cluster_u32(map_to_cta(smem_u32(tmem_holder), 0)) != tmem) {
-    flag_error(abort, kErrTmem);
-  }
-  __syncthreads();
-  const bool run = *abort == 0;
 
   if (warp >= 8) {
     regs_decrease<kCtlRegs>();
-    if (run && warp == kLoadWarp) {
-      if (lane == 0) run_producer(&tmap, p, smem_base, bars, rank, abort, issued, b, h, qq);
-    } else if (run && warp == kMmaWarp && rank == 0) {
+    if (warp == kLoadWarp) {
+      if (lane == 0) run_producer(&tmap, p, smem_base, bars, abort, issued, b, h, qp);
+    } else if (warp == kMmaWarp) {
       if (lane == 0) run_mma(p, smem_base, bars, abort, tmem);
     }
     __syncwarp();
   } else {
     regs_increase<kSoftmaxRegs>();
-    if (run) run_softmax(p, bars, abort, tmem, rank, warp >> 2, warp & 3, lane, b, h, qq);
+    run_softmax(p, bars, abort, tmem, warp >> 2, warp & 3, lane, b, h, qp);
   }
 
   tc_fence_before();
   __syncthreads();
-  if (rank == 0 && warp == kLoadWarp && lane == 0 && *abort) drain_producer(bars, issued);
-  cluster_sync();  // the partner's MMAs, loads and arrivals are all done
+  if (warp == kLoadWarp && lane == 0 && *abort) drain_producer(bars, issued);
   if (warp == kMmaWarp) {
     tc_fence_after();
-    tmem_dealloc_pair(tmem, kTmemCols);
+    tmem_dealloc(tmem, kTmemCols);
   }
 }
 
@@ -549,12 +459,12 @@ cudaError_t plan_attn_fwd(const void* qkv, void* out, int64_t batch, int64_t seq
   if (attr_err != cudaSuccess) return attr_err;
 
   // Packed buffer as a 3D tensor: x = channel (3D), y = token, z = batch.
-  // Boxes are 64 channels (128 bytes, the swizzle span) x 64 tokens.
+  // Boxes are 64 channels (128 bytes, the swizzle span) x 128 tokens.
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(3 * D), static_cast<cuuint64_t>(S),
                         static_cast<cuuint64_t>(batch)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(3 * D) * 2,
                            static_cast<cuuint64_t>(3 * D) * 2 * static_cast<cuuint64_t>(S)};
-  cuuint32_t box[3] = {64, 64, 1};
+  cuuint32_t box[3] = {64, kBM, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = encode(reinterpret_cast<CUtensorMap*>(plan->tmap), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
                       const_cast<void*>(qkv), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -566,11 +476,11 @@ cudaError_t plan_attn_fwd(const void* qkv, void* out, int64_t batch, int64_t seq
   plan->S = S;
   plan->heads = heads;
   plan->D = D;
-  plan->q_pairs = (S + kPairRows - 1) / kPairRows;  // CTA pairs per (batch, head)
+  plan->q_pairs = (S + 2 * kBM - 1) / (2 * kBM);
   plan->n_kv = (S + kBN - 1) / kBN;
   const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(kHD));
   plan->scale_log2 = sc * 1.4426950408889634f;
-  plan->grid = 2 * batch * heads * static_cast<int64_t>(plan->q_pairs);  // two CTAs per pair
+  plan->grid = batch * heads * static_cast<int64_t>(plan->q_pairs);
   return cudaSuccess;
 }
 
@@ -580,7 +490,7 @@ cudaError_t launch_attn_fwd(const AttnPlan& plan, cudaStream_t stream, bool pdl)
   p.S = plan.S;
   p.heads = plan.heads;
   p.D = plan.D;
-  p.q_quads = plan.q_pairs;
+  p.q_pairs = plan.q_pairs;
   p.n_kv = plan.n_kv;
   p.scale_log2 = plan.scale_log2;
   CUtensorMap tmap;
@@ -591,15 +501,11 @@ cudaError_t launch_attn_fwd(const AttnPlan& plan, cudaStream_t stream, bool pdl)
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;  // CTA pairs
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 2 : 1;
+  cfg.numAttrs = pdl ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, attn_fwd_kernel, tmap, p);
 }
 

@@ -76,7 +76,7 @@ struct NormRopeParams {
   uint32_t stage_bytes;  // Q row + K row = 4 * D bytes
   double eps;
   double inv_d;
-  double freq[kPairs];   // per pair of a head: theta^(-2j/d_axis)
+  double freq_pi[kPairs];  // per pair of a head: theta^(-2j/d_axis) / pi
 };
 
 // Shared-memory layout behind the ring (offsets from the ring's end).
@@ -142,7 +142,7 @@ __device__ __forceinline__ void rotation(const NormRopeParams& p, int s, int pr,
   const int q = s / p.W;  // frame * H + row
   const int pos = pr < kRowAxisPair0 ? q / p.H : (pr < kColAxisPair0 ? q - (q / p.H) * p.H : s - q * p.W);
   double sd, cd;
-  sincos(static_cast<double>(pos) * p.freq[pr], &sd, &cd);
+  sincospi(static_cast<double>(pos) * p.freq_pi[pr], &sd, &cd);  // angle = pos * freq
   const float ch = __uint_as_float(__float_as_uint(static_cast<float>(cd)) & 0xFFFFFF00u);
   const float sh = __uint_as_float(__float_as_uint(static_cast<float>(sd)) & 0xFFFFFF00u);
   const float cl = static_cast<float>(cd - static_cast<double>(ch));
@@ -318,15 +318,16 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const __grid_
     }
 
     const double* part = &tail.partial[buf][4 * which];
-    const double rd = 1.0 / sqrt(((part[0] + part[1]) + (part[2] + part[3])) * p.inv_d + p.eps);
+    const double rd = rsqrt(((part[0] + part[1]) + (part[2] + part[3])) * p.inv_d + p.eps);
     const float r_hi = static_cast<float>(rd);
     const float r_lo = static_cast<float>(rd - static_cast<double>(r_hi));
     const uint64_t r2 = f2(r_hi, r_hi);
     uint16_t* x = p.qkv + tok * 3 * static_cast<int64_t>(p.D) + which * p.D;
 
-    // Pass A: y = bf16(x * g * r) for every pair held by this thread, with
-    // the exact rounding for the rare vectors near a rounding midpoint.
-    uint32_t y[VPT][4];
+    // Pass A: y = bf16(x * g * r) for every pair held by this thread (written
+    // over x), with the exact rounding for the rare vectors near a rounding
+    // midpoint.
+    uint32_t (&y)[VPT][4] = *reinterpret_cast<uint32_t(*)[VPT][4]>(v);
 #pragma unroll
     for (int k = 0; k < VPT; ++k) {
       const int vi = u + kRowThreads * k;
@@ -335,16 +336,19 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const __grid_
       const uint32_t xw[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
       const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
       uint32_t near = 0xFFFFFFFFu;
+      uint32_t yk[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) y[k][e] = norm_round(xw[e], gw[e], r2, near);
+      for (int e = 0; e < 4; ++e) yk[e] = norm_round(xw[e], gw[e], r2, near);
       if ((near & 0xFFF8u) == 0u || (near & 0xFFF80000u) == 0u) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const uint32_t lo = round_exact(bf16_lo(xw[e]) * bf16_lo(gw[e]), r_hi, r_lo);
           const uint32_t hi = round_exact(bf16_hi(xw[e]) * bf16_hi(gw[e]), r_hi, r_lo);
-          y[k][e] = lo | (hi << 16);
+          yk[e] = lo | (hi << 16);
         }
       }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) y[k][e] = yk[e];
     }
     // Pass B: rotate, two pair positions (of the 4 per thread) at a time so
     // that only their cos/sin operands are live.
@@ -431,7 +435,8 @@ cudaError_t launch_qk_norm_rope(void* qkv, int64_t batch, int32_t F, int32_t H, 
   for (int pr = 0; pr < kPairs; ++pr) {
     const int axis = pr < kRowAxisPair0 ? 0 : (pr < kColAxisPair0 ? 1 : 2);
     const int j = pr - (axis == 0 ? 0 : (axis == 1 ? kRowAxisPair0 : kColAxisPair0));
-    p.freq[pr] = std::pow(static_cast<double>(theta), -2.0 * j / static_cast<double>(split[axis]));
+    p.freq_pi[pr] =
+        std::pow(static_cast<double>(theta), -2.0 * j / static_cast<double>(split[axis])) / M_PI;
   }
   if (p.tokens == 0) return cudaSuccess;
   const uint32_t smem_bytes = p.stages * p.stage_bytes + static_cast<uint32_t>(sizeof(NormSmemTail));

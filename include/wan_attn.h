@@ -81,7 +81,7 @@ typedef enum {
 /* Static, human-readable text for a status code. Never NULL. */
 WAN_API const char* wan_status_string(int32_t status);
 
-/* Version of this ABI (bumped on any signature change). */
+/* Version of this ABI (bumped on any signature change or addition). */
 WAN_API int32_t wan_abi_version(void);
 
 /*
@@ -134,6 +134,22 @@ WAN_API int32_t wan_dit_attn(void* qkv, void* out, int64_t batch, int32_t F, int
  * NULL, WAN_ERR_LAUNCH when the synchronisation reports a CUDA error.
  */
 WAN_API int32_t wan_device_error(void* stream, int32_t* code);
+
+/*
+ * Self-test of failure detection. Launches the attention kernel exactly as
+ * wan_self_attention does, except that its producer starts no copies, so
+ * every bounded wait of the kernel runs out after `wait_limit_ns`
+ * (1e3 .. 2e9 ns). The kernel then records the timeout in its device error
+ * word, drains, releases its tensor memory and exits without touching `out`.
+ * Read the result with wan_device_error (expected: WAN_ERR_DEVICE_TIMEOUT with
+ * a nonzero site code); the CUDA context stays usable. This is how a stalled
+ * pipeline surfaces as an error instead of a hang (the vLLM-Omni recipe's
+ * rule that the backend raises rather than silently degrading).
+ * Arguments as for wan_self_attention; nothing is written to qkv or out.
+ */
+WAN_API int32_t wan_selftest_wait_timeout(const void* qkv, void* out, int64_t batch, int64_t seq_len,
+                                          int32_t heads, int32_t head_dim, int64_t wait_limit_ns,
+                                          void* stream);
 
 #ifdef __cplusplus
 }

@@ -39,7 +39,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings(lib):
-    assert lib.wan_abi_version() == 1
+    assert lib.wan_abi_version() == 2
     for code in range(10):
         assert lib.wan_status_string(code)
     assert lib.wan_status_string(99) == b"unknown status"
@@ -95,3 +95,10 @@ def test_valid_arguments_without_a_b200_fail_loudly(lib):
     assert st == 6  # WAN_ERR_UNSUPPORTED_DEVICE: no silent fallback
     with pytest.raises(TypeError):
         wan.self_attention(torch.zeros(1, 8, 384, dtype=torch.bfloat16), 1)
+
+
+def test_selftest_entry_point_validates_before_launch(lib):
+    # (qkv, out, batch, seq_len, heads, head_dim, wait_limit_ns)
+    assert lib.wan_selftest_wait_timeout(None, FAKE, 1, 8, 1, 128, 10**7, None) == 1
+    assert lib.wan_selftest_wait_timeout(FAKE, FAKE * 16, 1, 8, 1, 128, 10, None) == 5
+    assert lib.wan_selftest_wait_timeout(FAKE, FAKE * 16, 1, 8, 1, 64, 10**7, None) == 4

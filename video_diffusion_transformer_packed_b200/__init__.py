@@ -19,7 +19,7 @@ import threading
 from typing import Optional, Sequence
 
 __all__ = ["WanError", "load_library", "library_path", "qk_norm_rope", "self_attention",
-           "dit_attn", "device_error", "HEAD_DIM", "EPS", "THETA", "STATUS"]
+           "dit_attn", "device_error", "selftest_wait_timeout", "HEAD_DIM", "EPS", "THETA", "STATUS"]
 
 HEAD_DIM = 128
 EPS = 1e-6
@@ -69,6 +69,8 @@ def load_library() -> ctypes.CDLL:
             lib.wan_dit_attn.restype = I32
             lib.wan_device_error.argtypes = [P, ctypes.POINTER(I32)]
             lib.wan_device_error.restype = I32
+            lib.wan_selftest_wait_timeout.argtypes = [P, P, I64, I64, I32, I32, I64, P]
+            lib.wan_selftest_wait_timeout.restype = I32
             _lib = lib
     return _lib
 
@@ -157,6 +159,21 @@ def dit_attn(qkv, grid: Sequence[int], heads: int, gamma_q, gamma_k, out=None, e
                                        heads, HEAD_DIM, _bf16_cuda(gamma_q, "gamma_q"),
                                        _bf16_cuda(gamma_k, "gamma_k"), eps, theta, scale,
                                        _stream(stream)), "wan_dit_attn")
+    return out
+
+
+def selftest_wait_timeout(qkv, heads: int, out=None, wait_limit_ns: int = 20_000_000, stream=None):
+    """Launch the attention kernel with its loads suppressed so that its bounded
+    waits run out; read the outcome with device_error() (nonzero expected)."""
+    import torch
+    _check_packed(qkv, heads)
+    B, S, _ = qkv.shape
+    if out is None:
+        out = torch.empty((B, S, heads * HEAD_DIM), dtype=torch.bfloat16, device=qkv.device)
+    _check_out(out, qkv, heads)
+    _check(load_library().wan_selftest_wait_timeout(_bf16_cuda(qkv, "qkv"), _bf16_cuda(out, "out"), B, S,
+                                                    heads, HEAD_DIM, int(wait_limit_ns), _stream(stream)),
+           "wan_selftest_wait_timeout")
     return out
 
 

@@ -11,7 +11,7 @@
 
 namespace {
 
-constexpr int32_t kAbiVersion = 1;
+constexpr int32_t kAbiVersion = 2;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -159,6 +159,25 @@ int32_t wan_dit_attn(void* qkv, void* out, int64_t batch, int32_t F, int32_t H, 
     return WAN_ERR_LAUNCH;
   }
   if (wan::launch_attn_fwd(plan, st, true) != cudaSuccess) {
+    return WAN_ERR_LAUNCH;
+  }
+  return WAN_OK;
+}
+
+int32_t wan_selftest_wait_timeout(const void* qkv, void* out, int64_t batch, int64_t seq_len,
+                                  int32_t heads, int32_t head_dim, int64_t wait_limit_ns, void* stream) {
+  WAN_TRY(check_heads(heads, head_dim));
+  WAN_TRY(check_tokens(batch, seq_len, heads));
+  WAN_TRY(check_attn_args(qkv, out, batch, seq_len, heads, 0.f));
+  if (wait_limit_ns < 1000 || wait_limit_ns > 2000000000) return WAN_ERR_PARAM;
+  WAN_TRY(check_device());
+  (void)cudaGetLastError();
+  wan::AttnPlan plan;
+  if (wan::plan_attn_fwd(qkv, out, batch, seq_len, heads, 0.f, &plan) != cudaSuccess) {
+    return WAN_ERR_LAUNCH;
+  }
+  if (wan::launch_attn_fwd(plan, static_cast<cudaStream_t>(stream), false,
+                           static_cast<uint64_t>(wait_limit_ns), true) != cudaSuccess) {
     return WAN_ERR_LAUNCH;
   }
   return WAN_OK;

@@ -63,7 +63,7 @@ constexpr int kCtlRegs = 72;
 constexpr int kSoftmaxRegs = 216;
 static_assert(128 * kCtlRegs + 256 * kSoftmaxRegs <= kThreads * kLaunchRegs, "register split");
 constexpr uint32_t kTmemCols = 512;
-constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait (the default limit)
 constexpr float kRescaleThreshold = 8.0f;         // log2 of the largest tolerated growth
 
 // Shared memory map (offsets from a 1024-byte aligned base).
@@ -87,6 +87,8 @@ struct AttnParams {
   int32_t q_pairs;  // ceil(S / 256): CTAs per (batch, head)
   int32_t n_kv;     // ceil(S / 128)
   float scale_log2; // scale * log2(e)
+  uint64_t wait_ns; // limit of each pipeline wait
+  int32_t skip_loads;  // self-test: the producer starts no copies, so the waits run out
 };
 
 // Barrier addresses (32-bit shared-memory addresses, 8 bytes apart).
@@ -111,7 +113,9 @@ __device__ __forceinline__ void flag_error(volatile int* abort, int site) {
 __device__ void run_producer(const CUtensorMap* tmap, const AttnParams& p, uint32_t smem,
                              Bars bars, volatile int* abort, int* issued, int b, int h, int qp) {
   grid_dependency_wait();  // the packed buffer may still be written by the norm kernel
+  if (p.skip_loads) return;  // self-test of the bounded waits: nothing will arrive
   const int xq = h * kHD, xk = p.D + h * kHD, xv = 2 * p.D + h * kHD;
+  issued[kStages] = 1;  // the Q copies
   mbar_arrive_expect_tx(bars.q_full(), 2 * kTileBytes);
   for (int t = 0; t < 2; ++t) {
     for (int half = 0; half < 2; ++half) {
@@ -125,7 +129,7 @@ __device__ void run_producer(const CUtensorMap* tmap, const AttnParams& p, uint3
   for (int i = 0; i < items; ++i) {
     const int slot = i % kStages;
     const int use = i / kStages;
-    if (use > 0 && !mbar_wait(bars.kv_empty(slot), (use - 1) & 1, abort, kWaitLimitNs)) {
+    if (use > 0 && !mbar_wait(bars.kv_empty(slot), (use - 1) & 1, abort, p.wait_ns)) {
       ok = false;
       break;
     }
@@ -148,7 +152,9 @@ __device__ void drain_producer(Bars bars, const int* issued) {
       atomicOr(&g_attn_error_word, kErrDrain);
     }
   }
-  if (!mbar_wait(bars.q_full(), 0, nullptr, kWaitLimitNs)) atomicOr(&g_attn_error_word, kErrDrain);
+  if (issued[kStages] && !mbar_wait(bars.q_full(), 0, nullptr, kWaitLimitNs)) {
+    atomicOr(&g_attn_error_word, kErrDrain);
+  }
 }
 
 // -------------------------------------------------------------- MMA issuer
@@ -189,10 +195,10 @@ __device__ void run_mma(const AttnParams& p, uint32_t smem, Bars bars, volatile 
     }
   };
   auto wait_item = [&](int i) -> bool {
-    return mbar_wait(bars.kv_full(i % kStages), (i / kStages) & 1, abort, kWaitLimitNs);
+    return mbar_wait(bars.kv_full(i % kStages), (i / kStages) & 1, abort, p.wait_ns);
   };
 
-  bool ok = mbar_wait(bars.q_full(), 0, abort, kWaitLimitNs) && wait_item(0);
+  bool ok = mbar_wait(bars.q_full(), 0, abort, p.wait_ns) && wait_item(0);
   if (ok) {
     tc_fence_after();
     issue_qk(0, 0);
@@ -206,7 +212,7 @@ __device__ void run_mma(const AttnParams& p, uint32_t smem, Bars bars, volatile 
     const int iv = 2 * j + 1, ik = 2 * j + 2;
     const bool more = j + 1 < p.n_kv;
     const uint32_t acc = j > 0 ? 1u : 0u;
-    if (!wait_item(iv) || !mbar_wait(bars.p_full(0), j & 1, abort, kWaitLimitNs)) { ok = false; break; }
+    if (!wait_item(iv) || !mbar_wait(bars.p_full(0), j & 1, abort, p.wait_ns)) { ok = false; break; }
     tc_fence_after();
     issue_pv(0, iv % kStages, acc);
     if (more) {
@@ -215,7 +221,7 @@ __device__ void run_mma(const AttnParams& p, uint32_t smem, Bars bars, volatile 
       issue_qk(0, ik % kStages);
       mma_commit(bars.s_full(0));
     }
-    if (!mbar_wait(bars.p_full(1), j & 1, abort, kWaitLimitNs)) { ok = false; break; }
+    if (!mbar_wait(bars.p_full(1), j & 1, abort, p.wait_ns)) { ok = false; break; }
     tc_fence_after();
     issue_pv(1, iv % kStages, acc);
     mma_commit(bars.kv_empty(iv % kStages));
@@ -249,7 +255,7 @@ __device__ void run_softmax(const AttnParams& p, Bars bars, volatile int* abort,
 
 #pragma unroll 1
   for (int j = 0; j < p.n_kv; ++j) {
-    if (!mbar_wait(bars.s_full(t), j & 1, abort, kWaitLimitNs)) { ok = false; break; }
+    if (!mbar_wait(bars.s_full(t), j & 1, abort, p.wait_ns)) { ok = false; break; }
     tc_fence_after();
     uint32_t sr[128];  // raw fp32 scores of this thread's row
     tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(sr + 0));
@@ -327,7 +333,7 @@ __device__ void run_softmax(const AttnParams& p, Bars bars, volatile int* abort,
     flag_error(abort, kErrSoftmax);
     return;
   }
-  if (!mbar_wait(bars.o_full(t), 0, abort, kWaitLimitNs)) {
+  if (!mbar_wait(bars.o_full(t), 0, abort, p.wait_ns)) {
     flag_error(abort, kErrEpilogue);
     return;
   }
@@ -361,7 +367,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const Bars bars{smem_base + kOffBar};
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
-  int* issued = reinterpret_cast<int*>(smem + kOffMisc + 8);  // [kStages], producer-owned
+  int* issued = reinterpret_cast<int*>(smem + kOffMisc + 8);  // [kStages + 1], producer-owned
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -383,7 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(bars.drain(), 1);
     *abort = 0;
-    for (int s = 0; s < kStages; ++s) issued[s] = 0;
+    for (int s = 0; s <= kStages; ++s) issued[s] = 0;
     fence_mbar_init();
   }
   if (warp == kMmaWarp) {
@@ -484,7 +490,8 @@ cudaError_t plan_attn_fwd(const void* qkv, void* out, int64_t batch, int64_t seq
   return cudaSuccess;
 }
 
-cudaError_t launch_attn_fwd(const AttnPlan& plan, cudaStream_t stream, bool pdl) {
+cudaError_t launch_attn_fwd(const AttnPlan& plan, cudaStream_t stream, bool pdl, uint64_t wait_ns,
+                            bool skip_loads) {
   AttnParams p;
   p.out = static_cast<uint16_t*>(plan.out);
   p.S = plan.S;
@@ -493,6 +500,8 @@ cudaError_t launch_attn_fwd(const AttnPlan& plan, cudaStream_t stream, bool pdl)
   p.q_pairs = plan.q_pairs;
   p.n_kv = plan.n_kv;
   p.scale_log2 = plan.scale_log2;
+  p.wait_ns = wait_ns;
+  p.skip_loads = skip_loads ? 1 : 0;
   CUtensorMap tmap;
   memcpy(&tmap, plan.tmap, sizeof(tmap));
 

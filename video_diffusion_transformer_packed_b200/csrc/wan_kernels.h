@@ -28,8 +28,12 @@ cudaError_t plan_attn_fwd(const void* qkv, void* out, int64_t batch, int64_t seq
                           int32_t heads, float scale, AttnPlan* plan);
 
 // Flash attention over the packed buffer. `pdl` marks the launch as a
-// programmatic dependent of the previous kernel on the stream.
-cudaError_t launch_attn_fwd(const AttnPlan& plan, cudaStream_t stream, bool pdl);
+// programmatic dependent of the previous kernel on the stream; `wait_ns`
+// bounds every pipeline wait; `skip_loads` (self-test only) starts no copies,
+// so that the waits run out and the kernel reports a timeout.
+constexpr uint64_t kDefaultWaitNs = 1000000000ull;
+cudaError_t launch_attn_fwd(const AttnPlan& plan, cudaStream_t stream, bool pdl,
+                            uint64_t wait_ns = kDefaultWaitNs, bool skip_loads = false);
 
 // Synchronise the stream, then read and clear a kernel's device error word.
 cudaError_t read_and_clear_device_error(cudaStream_t stream, int32_t* code);

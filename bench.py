@@ -69,22 +69,33 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def sha256(path):
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()
+SM100_HDR = os.path.join(ROOT, "video_diffusion_transformer_packed_b200", "csrc", "sm100.cuh")
 
 
-def profiled_traffic(kernel: str, src: str):
-    """DRAM bytes per launch from the committed ncu summary of `kernel`, if the
-    summary was taken on the current kernel source; else None."""
-    for fn in sorted(os.listdir(os.path.join(ROOT, "profiles"))) if os.path.isdir(os.path.join(ROOT, "profiles")) else []:
+def kernel_sha256(src):
+    """sha256 of a kernel's source followed by the shared PTX-wrapper header:
+    both decide the compiled kernel."""
+    h = hashlib.sha256()
+    for path in (src, SM100_HDR):
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def profiled_traffic(kernel: str, src: str, tokens: int):
+    """DRAM bytes per launch for a launch over `tokens` tokens (batch x S), from
+    the committed ncu summary of `kernel` (bytes per token; both kernels move
+    a fixed number of bytes per token), if the summary was taken on the
+    current kernel source; else None."""
+    pdir = os.path.join(ROOT, "profiles")
+    for fn in sorted(os.listdir(pdir)) if os.path.isdir(pdir) else []:
         if not fn.startswith(kernel):
             continue
-        txt = open(os.path.join(ROOT, "profiles", fn)).read()
+        txt = open(os.path.join(pdir, fn)).read()
         m_sha = re.search(r"kernel_source_sha256\s*[:=]\s*([0-9a-f]{64})", txt)
-        m_tr = re.search(r"traffic_per_launch_bytes\s*[:=]\s*([0-9.eE+]+)", txt)
-        if m_sha and m_tr and m_sha.group(1) == sha256(src):
-            return float(m_tr.group(1))
+        m_tr = re.search(r"traffic_per_token_bytes\s*[:=]\s*([0-9.eE+]+)", txt)
+        if m_sha and m_tr and m_sha.group(1) == kernel_sha256(src):
+            return float(m_tr.group(1)) * tokens
     return None
 
 
@@ -345,7 +356,7 @@ def run_ours(args):
     roofline = {
         "kernel": "attn_fwd", "bound": "tensor", "achieved": attn_tflops, "peak": tensor_peak,
         "unit": "TFLOP/s", "frac": attn_tflops / tensor_peak,
-        "traffic": profiled_traffic("attn_fwd", ATTN_SRC),
+        "traffic": profiled_traffic("attn_fwd", ATTN_SRC, w.batch * w.seq_len),
         "peak_source": f"{peak_src} bf16 sustained (kernel timed inside seconds-long loops)",
         "frac_of_burst_peak": attn_tflops / peaks["bf16_tflops"],
         "algorithmic_flop_per_launch": w.attn_flop, "avg_launch_ms": t_attn,
@@ -353,7 +364,7 @@ def run_ours(args):
     norm_roofline = {
         "kernel": "qk_norm_rope", "bound": "hbm", "achieved": norm_gbs, "peak": peaks["hbm_gbs"],
         "unit": "GB/s", "frac": norm_gbs / peaks["hbm_gbs"],
-        "traffic": profiled_traffic("qk_norm_rope", NORM_SRC),
+        "traffic": profiled_traffic("qk_norm_rope", NORM_SRC, w.batch * w.seq_len),
         "algorithmic_bytes_per_launch": w.norm_rope_bytes, "avg_launch_ms": t_norm,
         "peak_source": f"{peak_src} copy bandwidth",
     }

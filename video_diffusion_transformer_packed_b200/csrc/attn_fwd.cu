@@ -65,12 +65,18 @@ static_assert(128 * kCtlRegs + 256 * kSoftmaxRegs <= kThreads * kLaunchRegs, "re
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait (the default limit)
 constexpr float kRescaleThreshold = 8.0f;         // log2 of the largest tolerated growth
+// P_t is handed to the MMA issuer in kPParts column blocks, each with its own
+// barrier: O_t += P_t V starts on the first keys while the softmax is still
+// exponentiating the last ones.
+constexpr int kPParts = 2;
+constexpr int kPairsPerPart = 64 / kPParts;  // bf16 pairs (TMEM columns) per block
+static_assert(kPParts == 1 || kPParts == 2 || kPParts == 4, "P blocks");
 
 // Shared memory map (offsets from a 1024-byte aligned base).
 constexpr int kOffQ = 0;                              // 2 tiles
 constexpr int kOffKV = kOffQ + 2 * kTileBytes;        // kStages tiles
 constexpr int kOffBar = kOffKV + kStages * kTileBytes;
-constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 2 + 1;  // q, kv full/empty, s, p, o, drain
+constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 * kPParts + 2 + 1;  // q, kv full/empty, s, p, o, drain
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + alignment slack
 
@@ -98,11 +104,13 @@ struct Bars {
   __device__ __forceinline__ uint32_t kv_full(int s) const { return base + 8 * (1 + s); }
   __device__ __forceinline__ uint32_t kv_empty(int s) const { return base + 8 * (1 + kStages + s); }
   __device__ __forceinline__ uint32_t s_full(int t) const { return base + 8 * (1 + 2 * kStages + t); }
-  __device__ __forceinline__ uint32_t p_full(int t) const { return base + 8 * (3 + 2 * kStages + t); }
-  __device__ __forceinline__ uint32_t o_full(int t) const { return base + 8 * (5 + 2 * kStages + t); }
-  __device__ __forceinline__ uint32_t drain() const { return base + 8 * (7 + 2 * kStages); }
+  __device__ __forceinline__ uint32_t p_full(int t, int part) const {
+    return base + 8 * (3 + 2 * kStages + t * kPParts + part);
+  }
+  __device__ __forceinline__ uint32_t o_full(int t) const { return base + 8 * (3 + 2 * kStages + 2 * kPParts + t); }
+  __device__ __forceinline__ uint32_t drain() const { return base + 8 * (5 + 2 * kStages + 2 * kPParts); }
 };
-static_assert(8 + 2 * kStages == kNumBars, "barrier count");
+static_assert(6 + 2 * kStages + 2 * kPParts == kNumBars, "barrier count");
 
 __device__ __forceinline__ void flag_error(volatile int* abort, int site) {
   *abort = 1;
@@ -165,70 +173,113 @@ __device__ void run_mma(const AttnParams& p, uint32_t smem, Bars bars, volatile 
   // Descriptors are built once; a step only adds a byte offset (in 16-byte
   // units) to the start-address field, which cannot carry out of its 14 bits
   // because shared-memory addresses stay below 2^18.
-  //
-  // S_t = Q_t K^T: K = 128 head dims in 8 steps of 16; each 64-dim half of a
-  // tile is one 128-byte-swizzled box, and a 16-element step inside a box
-  // advances the start address by 32 bytes.
   const uint64_t q_desc0 = smem_desc_sw128(smem + kOffQ, 16, 1024);
   const uint64_t k_desc0 = smem_desc_sw128(smem + kOffKV, 16, 1024);
   // V [key][dim] is an N-major B: 8-key groups 1024 bytes apart, the two
   // 64-dim halves one box (16 KB) apart; a 16-key step advances 2048 bytes.
   const uint64_t v_desc0 = smem_desc_sw128(smem + kOffKV, kBoxBytes, 1024);
 
-  auto issue_qk = [&](int t, int slot) {
+  // MMA steps [k0, k1) of one 128 x 128 x 128 product; a step is K = 16.
+  // S_t = Q_t K^T: each 64-dim half of a tile is one 128-byte-swizzled box,
+  // and a 16-element step inside a box advances the start address by 32 bytes.
+  auto qk_steps = [&](int t, int slot, int k0, int k1) {
     const uint32_t a0 = (t * kTileBytes) >> 4;
     const uint32_t b0 = (slot * kTileBytes) >> 4;
 #pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
+    for (int kk = k0; kk < k1; ++kk) {
       const uint32_t off = ((kk >> 2) * kBoxBytes + (kk & 3) * 32) >> 4;
       mma_ss(tmem + t * 128, desc_add(q_desc0, a0 + off), desc_add(k_desc0, b0 + off), kIdescQK,
              kk > 0 ? 1u : 0u);
     }
   };
   // O_t += P_t V: P_t (bf16, 64 TMEM columns over S_t) is the A operand.
-  auto issue_pv = [&](int t, int slot, uint32_t acc) {
+  auto pv_steps = [&](int t, int slot, int k0, int k1, uint32_t acc) {
     const uint32_t b0 = (slot * kTileBytes) >> 4;
 #pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
+    for (int kk = k0; kk < k1; ++kk) {
       mma_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, desc_add(v_desc0, b0 + kk * (2048 >> 4)),
              kIdescPV, kk > 0 ? 1u : acc);
     }
   };
-  auto wait_item = [&](int i) -> bool {
-    return mbar_wait(bars.kv_full(i % kStages), (i / kStages) & 1, abort, p.wait_ns);
+  // The tensor core's instruction queue holds little more than one MMA, so
+  // every barrier check between two groups of MMAs would leave it idle for a
+  // shared-memory round trip. Instead the next group's barrier is probed
+  // (non-blocking) just before the current group's last MMA, whose issue the
+  // thread waits for anyway; the blocking wait runs only when the probe
+  // found the phase still open.
+  auto ensure = [&](bool probed, uint32_t bar, uint32_t parity) -> bool {
+    if (!probed && !mbar_wait(bar, parity, abort, p.wait_ns)) return false;
+    tc_fence_after();
+    return true;
   };
+  constexpr int kStepsPerPart = 8 / kPParts;
+  auto kv_bar = [&](int i) { return bars.kv_full(i % kStages); };
+  auto kv_par = [&](int i) { return static_cast<uint32_t>((i / kStages) & 1); };
 
-  bool ok = mbar_wait(bars.q_full(), 0, abort, p.wait_ns) && wait_item(0);
+  bool ok = mbar_wait(bars.q_full(), 0, abort, p.wait_ns) && mbar_wait(kv_bar(0), 0, abort, p.wait_ns);
+  bool next_v = false, next_p = false;  // probes of V_j and P_0(j) part 0
   if (ok) {
     tc_fence_after();
-    issue_qk(0, 0);
+    qk_steps(0, 0, 0, 8);
     mma_commit(bars.s_full(0));
-    issue_qk(1, 0);
+    qk_steps(1, 0, 0, 7);
+    next_v = mbar_test(kv_bar(1), kv_par(1));
+    qk_steps(1, 0, 7, 8);
     mma_commit(bars.s_full(1));
     mma_commit(bars.kv_empty(0));
   }
 #pragma unroll 1
   for (int j = 0; j < p.n_kv && ok; ++j) {
     const int iv = 2 * j + 1, ik = 2 * j + 2;
+    const int sv = iv % kStages, sk = ik % kStages;
     const bool more = j + 1 < p.n_kv;
     const uint32_t acc = j > 0 ? 1u : 0u;
-    if (!wait_item(iv) || !mbar_wait(bars.p_full(0), j & 1, abort, p.wait_ns)) { ok = false; break; }
-    tc_fence_after();
-    issue_pv(0, iv % kStages, acc);
-    if (more) {
-      if (!wait_item(ik)) { ok = false; break; }
-      tc_fence_after();
-      issue_qk(0, ik % kStages);
-      mma_commit(bars.s_full(0));
+    const uint32_t pj = j & 1;
+    if (!ensure(next_v, kv_bar(iv), kv_par(iv)) || !ensure(next_p, bars.p_full(0, 0), pj)) {
+      ok = false;
+      break;
     }
-    if (!mbar_wait(bars.p_full(1), j & 1, abort, p.wait_ns)) { ok = false; break; }
-    tc_fence_after();
-    issue_pv(1, iv % kStages, acc);
-    mma_commit(bars.kv_empty(iv % kStages));
+    // O_0 += P_0 V_j, one block of P at a time.
+    bool probe = false;
+#pragma unroll
+    for (int part = 0; part < kPParts; ++part) {
+      if (part > 0 && !ensure(probe, bars.p_full(0, part), pj)) { ok = false; break; }
+      const int k0 = part * kStepsPerPart, k1 = k0 + kStepsPerPart;
+      pv_steps(0, sv, k0, k1 - 1, acc);
+      probe = part + 1 < kPParts ? mbar_test(bars.p_full(0, part + 1), pj)
+                                 : (more ? mbar_test(kv_bar(ik), kv_par(ik)) : true);
+      pv_steps(0, sv, k1 - 1, k1, acc);
+    }
+    if (!ok) break;
     if (more) {
-      issue_qk(1, ik % kStages);
+      // S_0 = Q_0 K_{j+1}^T
+      if (!ensure(probe, kv_bar(ik), kv_par(ik))) { ok = false; break; }
+      qk_steps(0, sk, 0, 7);
+      probe = mbar_test(bars.p_full(1, 0), pj);
+      qk_steps(0, sk, 7, 8);
+      mma_commit(bars.s_full(0));
+    } else {
+      probe = mbar_test(bars.p_full(1, 0), pj);
+    }
+    // O_1 += P_1 V_j
+#pragma unroll
+    for (int part = 0; part < kPParts; ++part) {
+      if (!ensure(probe, bars.p_full(1, part), pj)) { ok = false; break; }
+      const int k0 = part * kStepsPerPart, k1 = k0 + kStepsPerPart;
+      pv_steps(1, sv, k0, k1 - 1, acc);
+      probe = part + 1 < kPParts ? mbar_test(bars.p_full(1, part + 1), pj) : false;
+      pv_steps(1, sv, k1 - 1, k1, acc);
+    }
+    if (!ok) break;
+    mma_commit(bars.kv_empty(sv));
+    if (more) {
+      // S_1 = Q_1 K_{j+1}^T; probe what the next iteration starts with.
+      qk_steps(1, sk, 0, 7);
+      next_v = mbar_test(kv_bar(iv + 2), kv_par(iv + 2));
+      next_p = mbar_test(bars.p_full(0, 0), pj ^ 1u);
+      qk_steps(1, sk, 7, 8);
       mma_commit(bars.s_full(1));
-      mma_commit(bars.kv_empty(ik % kStages));
+      mma_commit(bars.kv_empty(sk));
     }
   }
   if (ok) {
@@ -307,11 +358,11 @@ __device__ void run_softmax(const AttnParams& p, Bars bars, volatile int* abort,
     const uint64_t negm2 = f2(-m_run, -m_run);
     uint64_t sum2[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};  // 4 chains
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      uint32_t pk[32];
+    for (int part = 0; part < kPParts; ++part) {
+      uint32_t pk[kPairsPerPart];
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const int pe = 32 * half + e;  // pair index: columns 2pe, 2pe+1
+      for (int e = 0; e < kPairsPerPart; ++e) {
+        const int pe = kPairsPerPart * part + e;  // pair index: columns 2pe, 2pe+1
         const uint64_t x2 = fma2(f2(__uint_as_float(sr[2 * pe]), __uint_as_float(sr[2 * pe + 1])), sl2_2, negm2);
         float x0, x1;
         f2_split(x2, x0, x1);
@@ -319,15 +370,21 @@ __device__ void run_softmax(const AttnParams& p, Bars bars, volatile int* abort,
         sum2[e & 3] = add2(sum2[e & 3], f2(p0, p1));
         pk[e] = pack_bf16x2(p0, p1);
       }
-      tmem_st32(tS + 32 * half, pk);
+      if constexpr (kPairsPerPart == 64) {
+        tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(pk));
+        tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(pk + 32));
+      } else if constexpr (kPairsPerPart == 32) {
+        tmem_st32(tS + 32 * part, *reinterpret_cast<uint32_t(*)[32]>(pk));
+      } else {
+        tmem_st16(tS + 16 * part, *reinterpret_cast<uint32_t(*)[16]>(pk));
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bars.p_full(t, part));
     }
     float sum_lo, sum_hi;
     f2_split(add2(add2(sum2[0], sum2[1]), add2(sum2[2], sum2[3])), sum_lo, sum_hi);
-    const float sum = sum_lo + sum_hi;
-    tmem_wait_st();
-    tc_fence_before();
-    mbar_arrive(bars.p_full(t));
-    l_run += sum;
+    l_run += sum_lo + sum_hi;
   }
   if (!ok) {
     flag_error(abort, kErrSoftmax);
@@ -384,7 +441,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(bars.s_full(t), 1);
-      mbar_init(bars.p_full(t), 128);
+      for (int part = 0; part < kPParts; ++part) mbar_init(bars.p_full(t, part), 128);
       mbar_init(bars.o_full(t), 1);
     }
     mbar_init(bars.drain(), 1);

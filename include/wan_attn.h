@@ -38,7 +38,8 @@
  * j-th pair of an axis of width d_a has angle pos * theta^(-2j/d_a).
  *
  * Ownership and execution: the caller owns every buffer; the library
- * allocates no device memory. Calls are asynchronous on `stream` (a
+ * allocates no device memory (wan_dit_attn_host keeps two copy streams and
+ * a pool of events per device). Calls are asynchronous on `stream` (a
  * cudaStream_t; NULL is the legacy default stream) and do not synchronise.
  * Arguments are validated before anything is launched; on any error status
  * nothing has been launched and no buffer has been written.
@@ -71,8 +72,16 @@ typedef enum {
   WAN_ERR_UNSUPPORTED_DEVICE = 6, /* current device is not compute capability 10.0 */
   WAN_ERR_LAUNCH = 7,             /* the CUDA runtime rejected a launch */
   WAN_ERR_DEVICE_TIMEOUT = 8,     /* a kernel's bounded wait gave up (see wan_device_error) */
-  WAN_ERR_ALIAS = 9               /* out overlaps qkv */
+  WAN_ERR_ALIAS = 9,              /* out overlaps qkv */
+  WAN_ERR_MEMORY_KIND = 10        /* a host buffer is not page-locked, or a device buffer
+                                     is not memory of the current device */
 } wan_status;
+
+/* Default head-chunk size of wan_dit_attn_host's pipeline. */
+#define WAN_HOST_HEADS_PER_CHUNK 8
+/* Largest number of (batch element, head chunk) pieces one wan_dit_attn_host
+ * call is cut into. */
+#define WAN_HOST_MAX_PIECES 4096
 
 /* Largest head count accepted (hidden width 64*128 = 8192). */
 #define WAN_MAX_HEADS 64
@@ -125,6 +134,45 @@ WAN_API int32_t wan_self_attention(const void* qkv, void* out, int64_t batch, in
 WAN_API int32_t wan_dit_attn(void* qkv, void* out, int64_t batch, int32_t F, int32_t H, int32_t W,
                      int32_t heads, int32_t head_dim, const void* gamma_q, const void* gamma_k,
                      float eps, float theta, float scale, void* stream);
+
+/*
+ * (1) then (2) for packed QKV and output that live in HOST memory: the call
+ * a user with host-resident activations makes. Copies and kernels overlap
+ * chunk by chunk, because PCIe, not the kernels, bounds this step:
+ *  - per batch element, the Q|K channels of every token are copied first
+ *    (the RMS of (1) runs over all heads of a token), then (1) runs on that
+ *    batch element;
+ *  - V follows in chunks of heads_per_chunk heads, and (2) for a head chunk
+ *    starts as soon as its V chunk has arrived;
+ *  - each head chunk of `out` is copied back while later chunks compute.
+ * qkv_host  page-locked host memory (cudaHostAlloc / cudaHostRegister), bf16
+ *           [batch][F*H*W][3*heads*128]; only read.
+ * out_host  page-locked host memory, bf16 [batch][F*H*W][heads*128]; written.
+ * qkv_dev   device memory of the current device, same shape as qkv_host:
+ *           receives the copy and is normalised in place (left holding the
+ *           normalised Q|K and V).
+ * out_dev   device memory of the current device, same shape as out_host,
+ *           must not overlap qkv_dev.
+ * heads_per_chunk  1..heads, or 0 for WAN_HOST_HEADS_PER_CHUNK (capped at
+ *           heads); batch * ceil(heads/heads_per_chunk) <= WAN_HOST_MAX_PIECES.
+ * Other arguments as for wan_dit_attn. Device pointers 16-byte aligned.
+ * Execution: asynchronous and ordered on `stream`: the copies into qkv_dev
+ * start after the work enqueued on `stream` before this call, and work
+ * enqueued on `stream` after it runs once out_host is written (synchronise
+ * `stream` before reading out_host on the host). The library keeps two
+ * internal streams per device for the copies; concurrent calls on one device
+ * are serialised while they are enqueued.
+ * Errors: argument errors return before anything is enqueued, as for the other
+ * calls; WAN_ERR_MEMORY_KIND when a host buffer is not page-locked or a device
+ * buffer is not memory of the current device; WAN_ERR_LAUNCH when the runtime
+ * rejects a copy or launch while enqueueing (part of the step may then be
+ * enqueued already).
+ */
+WAN_API int32_t wan_dit_attn_host(const void* qkv_host, void* out_host, void* qkv_dev, void* out_dev,
+                                  int64_t batch, int32_t F, int32_t H, int32_t W, int32_t heads,
+                                  int32_t head_dim, const void* gamma_q, const void* gamma_k,
+                                  float eps, float theta, float scale, int32_t heads_per_chunk,
+                                  void* stream);
 
 /*
  * Synchronises `stream`, then reads and clears the device-side error word

@@ -29,7 +29,7 @@ def declared_functions():
 
 def test_header_declares_the_three_entry_points():
     names = declared_functions()
-    for n in ("wan_qk_norm_rope", "wan_self_attention", "wan_dit_attn"):
+    for n in ("wan_qk_norm_rope", "wan_self_attention", "wan_dit_attn", "wan_dit_attn_host"):
         assert n in names
 
 
@@ -39,8 +39,8 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings(lib):
-    assert lib.wan_abi_version() == 2
-    for code in range(10):
+    assert lib.wan_abi_version() == 3
+    for code in range(11):
         assert lib.wan_status_string(code)
     assert lib.wan_status_string(99) == b"unknown status"
 
@@ -102,3 +102,32 @@ def test_selftest_entry_point_validates_before_launch(lib):
     assert lib.wan_selftest_wait_timeout(None, FAKE, 1, 8, 1, 128, 10**7, None) == 1
     assert lib.wan_selftest_wait_timeout(FAKE, FAKE * 16, 1, 8, 1, 128, 10, None) == 5
     assert lib.wan_selftest_wait_timeout(FAKE, FAKE * 16, 1, 8, 1, 64, 10**7, None) == 4
+
+
+def test_host_pipeline_validates_before_touching_memory(lib):
+    # (qkv_host, out_host, qkv_dev, out_dev, batch, F, H, W, heads, head_dim, gq, gk, eps, theta,
+    #  scale, heads_per_chunk)
+    ok = (FAKE * 64, FAKE * 128, FAKE, FAKE * 16, 1, 2, 2, 2, 4, 128, FAKE, FAKE, 1e-6, 1e4, 0.0, 0)
+
+    def call(**kw):
+        a = list(ok)
+        names = ["qh", "oh", "qd", "od", "b", "F", "H", "W", "heads", "hd", "gq", "gk", "eps", "theta",
+                 "scale", "hc"]
+        for k, v in kw.items():
+            a[names.index(k)] = v
+        return lib.wan_dit_attn_host(*a, None)
+
+    assert call(qh=None) == 1
+    assert call(oh=None) == 1
+    assert call(qd=None) == 1
+    assert call(qd=FAKE + 8) == 2
+    assert call(hd=64) == 4
+    assert call(heads=0) == 3
+    assert call(eps=0.0) == 5
+    assert call(od=FAKE + 64) == 9  # out_dev overlaps qkv_dev
+    assert call(hc=-1) == 5
+    assert call(hc=5) == 5  # more than heads
+    assert call(b=5000, hc=1, od=2**40) == 3  # more pieces than the pipeline takes
+    import torch
+    if not torch.cuda.is_available():
+        assert call() == 6  # valid arguments, no B200: fails loudly

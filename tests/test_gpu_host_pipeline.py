@@ -1,0 +1,115 @@
+"""The host-buffer entry point wan_dit_attn_host: the pipelined step (strided
+host->device copies of Q|K and of V head chunks, per-batch norm+RoPE, attention
+per head chunk, device->host copies of the output) gives the same bits as the
+device-resident wan_dit_attn, for every chunking, ragged shapes included; it
+leaves qkv_host untouched, leaves the normalised buffer in qkv_dev, orders
+itself on the caller's stream, and refuses pageable host memory."""
+import math
+
+import pytest
+import torch
+
+import oracle
+import video_diffusion_transformer_packed_b200 as wan
+import wan_inputs as wi
+from video_diffusion_transformer_packed_b200 import build as wan_build
+from helpers import assert_attention_close
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    wan_build.build()
+
+
+def _device_reference(qkv, w, gq, gk):
+    d = qkv.cuda()
+    out = wan.dit_attn(d, w.grid, w.heads, gq, gk)
+    torch.cuda.synchronize()
+    return d, out
+
+
+def _pinned(t):
+    return t.contiguous().pin_memory()
+
+
+# (grid, heads, batch): the tiny Wan grid, a ragged S with a head count that
+# no chunk size divides, and the A14B head count at batch 2 (CFG)
+CASES = [((5, 8, 8), 12, 1), ((2, 10, 13), 7, 2), ((1, 9, 29), 40, 2)]
+
+
+@pytest.mark.parametrize("grid,heads,batch", CASES)
+@pytest.mark.parametrize("hc", [0, 1, 3, 8, 64])
+def test_host_pipeline_equals_device_path(grid, heads, batch, hc):
+    if hc > heads:
+        hc = heads
+    w = wi.Workload("case", batch, grid, heads)
+    qkv, gq, gk = wi.inputs_for(w, seed=11)
+    gq, gk = gq.cuda(), gk.cuda()
+    ref_qkv, ref_out = _device_reference(qkv, w, gq, gk)
+    qkv_h = _pinned(qkv)
+    keep = qkv_h.clone()
+    qkv_d = torch.full_like(ref_qkv, float("nan"))
+    out_d = torch.full_like(ref_out, float("nan"))
+    out_h = wan.dit_attn_host(qkv_h, w.grid, w.heads, gq, gk, qkv_dev=qkv_d, out_dev=out_d,
+                              heads_per_chunk=hc)
+    torch.cuda.synchronize()
+    assert wan.device_error() == 0
+    assert torch.equal(out_h.view(torch.int16), ref_out.cpu().view(torch.int16))
+    assert torch.equal(qkv_d.view(torch.int16), ref_qkv.view(torch.int16))
+    assert torch.equal(qkv_h.view(torch.int16), keep.view(torch.int16))  # input only read
+
+
+def test_host_pipeline_matches_oracle_tiny():
+    w = wi.WORKLOADS[0]
+    qkv, gq, gk = wi.inputs_for(w, seed=12)
+    out_h = wan.dit_attn_host(_pinned(qkv), w.grid, w.heads, gq.cuda(), gk.cuda())
+    torch.cuda.synchronize()
+    normed = oracle.qk_norm_rope(qkv, w.grid, w.heads, gq, gk, wi.EPS, wi.THETA)
+    ref = oracle.attention_full(normed, w.heads, 1.0 / math.sqrt(wi.HEAD_DIM))
+    assert_attention_close(out_h.view(1, w.seq_len, w.heads, wi.HEAD_DIM), ref, "host pipeline vs oracle")
+
+
+def test_host_pipeline_is_ordered_on_a_side_stream():
+    """Back-to-back calls on one non-default stream, reusing the device buffers:
+    each call waits for the previous one's copies, and a later kernel on the
+    stream sees the output written."""
+    w = wi.Workload("case", 2, (2, 10, 13), 7)
+    gq_h, gk_h = wi.gammas(w.heads)
+    gq, gk = gq_h.cuda(), gk_h.cuda()
+    s = torch.cuda.Stream()
+    qkv_d = torch.empty((w.batch, w.seq_len, 3 * w.dim), dtype=torch.bfloat16, device="cuda")
+    out_d = torch.empty((w.batch, w.seq_len, w.dim), dtype=torch.bfloat16, device="cuda")
+    outs, refs = [], []
+    for seed in (21, 22, 23):
+        qkv = wi.packed_qkv(w.batch, w.seq_len, w.heads, seed=seed)
+        _, ref = _device_reference(qkv, w, gq, gk)
+        refs.append(ref.cpu())
+        outs.append(wan.dit_attn_host(_pinned(qkv), w.grid, w.heads, gq, gk, qkv_dev=qkv_d,
+                                      out_dev=out_d, heads_per_chunk=3, stream=s))
+    s.synchronize()
+    for o, r in zip(outs, refs):
+        assert torch.equal(o.view(torch.int16), r.view(torch.int16))
+
+
+def test_host_pipeline_refuses_pageable_or_foreign_memory():
+    w = wi.WORKLOADS[0]
+    qkv, gq, gk = wi.inputs_for(w, seed=13)
+    gq, gk = gq.cuda(), gk.cuda()
+    with pytest.raises(TypeError):
+        wan.dit_attn_host(qkv, w.grid, w.heads, gq, gk)  # pageable: refused by the binding
+    lib = wan.load_library()
+    qkv_d = qkv.cuda()
+    out_d = torch.empty((1, w.seq_len, w.dim), dtype=torch.bfloat16, device="cuda")
+    out_pageable = torch.empty((1, w.seq_len, w.dim), dtype=torch.bfloat16)
+    args = [qkv.data_ptr(), out_pageable.data_ptr(), qkv_d.data_ptr(), out_d.data_ptr(), 1, *w.grid,
+            w.heads, 128, gq.data_ptr(), gk.data_ptr(), wi.EPS, wi.THETA, 0.0, 0, None]
+    assert lib.wan_dit_attn_host(*args) == 10  # pageable host memory
+    qkv_h, out_h = _pinned(qkv), _pinned(out_pageable)
+    args[0], args[1] = qkv_h.data_ptr(), out_h.data_ptr()
+    args[2] = qkv_h.data_ptr()  # a host buffer where device memory is required
+    assert lib.wan_dit_attn_host(*args) == 10
+    args[2] = qkv_d.data_ptr()
+    assert lib.wan_dit_attn_host(*args) == 0
+    torch.cuda.synchronize()

@@ -19,14 +19,16 @@ import threading
 from typing import Optional, Sequence
 
 __all__ = ["WanError", "load_library", "library_path", "qk_norm_rope", "self_attention",
-           "dit_attn", "device_error", "selftest_wait_timeout", "HEAD_DIM", "EPS", "THETA", "STATUS"]
+           "dit_attn", "dit_attn_host", "device_error", "selftest_wait_timeout", "HEAD_DIM", "EPS",
+           "THETA", "STATUS"]
 
 HEAD_DIM = 128
 EPS = 1e-6
 THETA = 10000.0
 STATUS = {0: "WAN_OK", 1: "WAN_ERR_NULL", 2: "WAN_ERR_ALIGN", 3: "WAN_ERR_SHAPE",
           4: "WAN_ERR_HEAD_DIM", 5: "WAN_ERR_PARAM", 6: "WAN_ERR_UNSUPPORTED_DEVICE",
-          7: "WAN_ERR_LAUNCH", 8: "WAN_ERR_DEVICE_TIMEOUT", 9: "WAN_ERR_ALIAS"}
+          7: "WAN_ERR_LAUNCH", 8: "WAN_ERR_DEVICE_TIMEOUT", 9: "WAN_ERR_ALIAS",
+          10: "WAN_ERR_MEMORY_KIND"}
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "_lib", "libwanattn.so")
@@ -71,6 +73,9 @@ def load_library() -> ctypes.CDLL:
             lib.wan_device_error.restype = I32
             lib.wan_selftest_wait_timeout.argtypes = [P, P, I64, I64, I32, I32, I64, P]
             lib.wan_selftest_wait_timeout.restype = I32
+            lib.wan_dit_attn_host.argtypes = [P, P, P, P, I64, I32, I32, I32, I32, I32, P, P, F, F, F,
+                                              I32, P]
+            lib.wan_dit_attn_host.restype = I32
             _lib = lib
     return _lib
 
@@ -160,6 +165,49 @@ def dit_attn(qkv, grid: Sequence[int], heads: int, gamma_q, gamma_k, out=None, e
                                        _bf16_cuda(gamma_k, "gamma_k"), eps, theta, scale,
                                        _stream(stream)), "wan_dit_attn")
     return out
+
+
+def _bf16_pinned(t, name: str) -> int:
+    import torch
+    if t.dtype != torch.bfloat16 or t.is_cuda or not t.is_contiguous() or not t.is_pinned():
+        raise TypeError(f"{name} must be a contiguous bfloat16 tensor in page-locked host memory")
+    return t.data_ptr()
+
+
+def dit_attn_host(qkv_host, grid: Sequence[int], heads: int, gamma_q, gamma_k, out_host=None,
+                  qkv_dev=None, out_dev=None, heads_per_chunk: int = 0, eps: float = EPS,
+                  theta: float = THETA, scale: float = 0.0, stream=None):
+    """The step for packed qkv in page-locked host memory: host->device copies,
+    qk_norm_rope, self_attention and the device->host copy of the output,
+    overlapped chunk by chunk inside the library. qkv_dev / out_dev are the
+    device buffers it runs through (allocated on the current device when not
+    given); qkv_host is only read. Asynchronous on `stream`: synchronise it
+    before reading out_host."""
+    import torch
+    F, H, W = grid
+    _check_packed(qkv_host, heads, grid)
+    _check_gamma(gamma_q, heads, "gamma_q")
+    _check_gamma(gamma_k, heads, "gamma_k")
+    B, S, _ = qkv_host.shape
+    dev = gamma_q.device
+    if out_host is None:
+        out_host = torch.empty((B, S, heads * HEAD_DIM), dtype=torch.bfloat16).pin_memory()
+    if qkv_dev is None:
+        qkv_dev = torch.empty(qkv_host.shape, dtype=torch.bfloat16, device=dev)
+    if out_dev is None:
+        out_dev = torch.empty((B, S, heads * HEAD_DIM), dtype=torch.bfloat16, device=dev)
+    _check_out(out_host, qkv_host, heads)
+    _check_packed(qkv_dev, heads, grid)
+    if tuple(qkv_dev.shape) != tuple(qkv_host.shape):
+        raise ValueError("qkv_dev must have the shape of qkv_host")
+    _check_out(out_dev, qkv_host, heads)
+    _check(load_library().wan_dit_attn_host(_bf16_pinned(qkv_host, "qkv_host"),
+                                            _bf16_pinned(out_host, "out_host"),
+                                            _bf16_cuda(qkv_dev, "qkv_dev"), _bf16_cuda(out_dev, "out_dev"),
+                                            B, F, H, W, heads, HEAD_DIM, _bf16_cuda(gamma_q, "gamma_q"),
+                                            _bf16_cuda(gamma_k, "gamma_k"), eps, theta, scale,
+                                            int(heads_per_chunk), _stream(stream)), "wan_dit_attn_host")
+    return out_host
 
 
 def selftest_wait_timeout(qkv, heads: int, out=None, wait_limit_ns: int = 20_000_000, stream=None):

@@ -11,7 +11,7 @@
 
 namespace {
 
-constexpr int32_t kAbiVersion = 2;
+constexpr int32_t kAbiVersion = 3;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -78,6 +78,31 @@ int32_t check_attn_args(const void* qkv, const void* out, int64_t batch, int64_t
   return WAN_OK;
 }
 
+// Host buffers must be page-locked (pinned or registered) so that the copies
+// run asynchronously; device buffers must be memory of the current device.
+int32_t check_memory_kind(const void* host_in, const void* host_out, const void* dev_a,
+                          const void* dev_b) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return WAN_ERR_UNSUPPORTED_DEVICE;
+  for (const void* p : {host_in, host_out}) {
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return WAN_ERR_MEMORY_KIND;
+    }
+    if (at.type != cudaMemoryTypeHost) return WAN_ERR_MEMORY_KIND;
+  }
+  for (const void* p : {dev_a, dev_b}) {
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return WAN_ERR_MEMORY_KIND;
+    }
+    if (at.type != cudaMemoryTypeDevice || at.device != dev) return WAN_ERR_MEMORY_KIND;
+  }
+  return WAN_OK;
+}
+
 #define WAN_TRY(expr)          \
   do {                         \
     const int32_t _s = (expr); \
@@ -100,6 +125,8 @@ const char* wan_status_string(int32_t status) {
     case WAN_ERR_LAUNCH: return "the CUDA runtime rejected a launch";
     case WAN_ERR_DEVICE_TIMEOUT: return "a bounded wait inside the attention kernel gave up";
     case WAN_ERR_ALIAS: return "out overlaps qkv";
+    case WAN_ERR_MEMORY_KIND:
+      return "a host buffer is not page-locked, or a device buffer is not memory of the current device";
     default: return "unknown status";
   }
 }
@@ -159,6 +186,46 @@ int32_t wan_dit_attn(void* qkv, void* out, int64_t batch, int32_t F, int32_t H, 
     return WAN_ERR_LAUNCH;
   }
   if (wan::launch_attn_fwd(plan, st, true) != cudaSuccess) {
+    return WAN_ERR_LAUNCH;
+  }
+  return WAN_OK;
+}
+
+int32_t wan_dit_attn_host(const void* qkv_host, void* out_host, void* qkv_dev, void* out_dev,
+                          int64_t batch, int32_t F, int32_t H, int32_t W, int32_t heads,
+                          int32_t head_dim, const void* gamma_q, const void* gamma_k, float eps,
+                          float theta, float scale, int32_t heads_per_chunk, void* stream) {
+  int64_t S = 0;
+  WAN_TRY(check_heads(heads, head_dim));
+  WAN_TRY(check_grid(batch, F, H, W, heads, &S));
+  if (!qkv_host || !out_host) return WAN_ERR_NULL;
+  WAN_TRY(check_norm_args(qkv_dev, gamma_q, gamma_k, eps, theta));
+  WAN_TRY(check_attn_args(qkv_dev, out_dev, batch, S, heads, scale));
+  if (heads_per_chunk < 0 || heads_per_chunk > heads) return WAN_ERR_PARAM;
+  const int32_t hc = heads_per_chunk > 0 ? heads_per_chunk
+                                         : (heads < WAN_HOST_HEADS_PER_CHUNK ? heads : WAN_HOST_HEADS_PER_CHUNK);
+  if (batch * ((heads + hc - 1) / hc) > WAN_HOST_MAX_PIECES) return WAN_ERR_SHAPE;
+  WAN_TRY(check_device());
+  WAN_TRY(check_memory_kind(qkv_host, out_host, qkv_dev, out_dev));
+  (void)cudaGetLastError();
+  wan::HostStep step;
+  step.qkv_host = qkv_host;
+  step.out_host = out_host;
+  step.qkv_dev = qkv_dev;
+  step.out_dev = out_dev;
+  step.batch = batch;
+  step.S = S;
+  step.F = F;
+  step.H = H;
+  step.W = W;
+  step.heads = heads;
+  step.heads_per_chunk = hc;
+  step.gamma_q = gamma_q;
+  step.gamma_k = gamma_k;
+  step.eps = eps;
+  step.theta = theta;
+  step.scale = scale;
+  if (wan::enqueue_dit_attn_host(step, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
     return WAN_ERR_LAUNCH;
   }
   return WAN_OK;

@@ -92,6 +92,7 @@ struct AttnParams {
   int32_t D;
   int32_t q_pairs;  // ceil(S / 256): CTAs per (batch, head)
   int32_t n_kv;     // ceil(S / 128)
+  int32_t b0, h0, nh;  // this launch covers batches [b0, ...) and heads [h0, h0 + nh)
   float scale_log2; // scale * log2(e)
   uint64_t wait_ns; // limit of each pipeline wait
   int32_t skip_loads;  // self-test: the producer starts no copies, so the waits run out
@@ -430,8 +431,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
   const int qp = blockIdx.x % p.q_pairs;
   const int bh = blockIdx.x / p.q_pairs;
-  const int b = bh / p.heads;
-  const int h = bh % p.heads;
+  const int b = p.b0 + bh / p.nh;
+  const int h = p.h0 + bh % p.nh;
 
   if (threadIdx.x == 0) {
     mbar_init(bars.q_full(), 1);
@@ -543,7 +544,10 @@ cudaError_t plan_attn_fwd(const void* qkv, void* out, int64_t batch, int64_t seq
   plan->n_kv = (S + kBN - 1) / kBN;
   const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(kHD));
   plan->scale_log2 = sc * 1.4426950408889634f;
-  plan->grid = batch * heads * static_cast<int64_t>(plan->q_pairs);
+  plan->b0 = 0;
+  plan->nb = static_cast<int32_t>(batch);
+  plan->h0 = 0;
+  plan->nh = heads;
   return cudaSuccess;
 }
 
@@ -556,6 +560,9 @@ cudaError_t launch_attn_fwd(const AttnPlan& plan, cudaStream_t stream, bool pdl,
   p.D = plan.D;
   p.q_pairs = plan.q_pairs;
   p.n_kv = plan.n_kv;
+  p.b0 = plan.b0;
+  p.h0 = plan.h0;
+  p.nh = plan.nh;
   p.scale_log2 = plan.scale_log2;
   p.wait_ns = wait_ns;
   p.skip_loads = skip_loads ? 1 : 0;
@@ -563,7 +570,12 @@ cudaError_t launch_attn_fwd(const AttnPlan& plan, cudaStream_t stream, bool pdl,
   memcpy(&tmap, plan.tmap, sizeof(tmap));
 
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(plan.grid));
+  const int64_t grid = static_cast<int64_t>(plan.nb) * plan.nh * plan.q_pairs;
+  if (plan.nb < 1 || plan.nh < 1 || plan.h0 < 0 || plan.b0 < 0 || plan.h0 + plan.nh > plan.heads ||
+      grid > INT32_MAX) {
+    return cudaErrorInvalidValue;
+  }
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = stream;

@@ -21,7 +21,10 @@ struct AttnPlan {
   void* out;
   int32_t S, heads, D, q_pairs, n_kv;
   float scale_log2;
-  int64_t grid;
+  // The (batch, head) block a launch covers: batches [b0, b0 + nb), heads
+  // [h0, h0 + nh). plan_attn_fwd sets the whole buffer; a pipelined caller
+  // narrows a copy of the plan per launch.
+  int32_t b0, nb, h0, nh;
 };
 
 cudaError_t plan_attn_fwd(const void* qkv, void* out, int64_t batch, int64_t seq_len,
@@ -34,6 +37,23 @@ cudaError_t plan_attn_fwd(const void* qkv, void* out, int64_t batch, int64_t seq
 constexpr uint64_t kDefaultWaitNs = 1000000000ull;
 cudaError_t launch_attn_fwd(const AttnPlan& plan, cudaStream_t stream, bool pdl,
                             uint64_t wait_ns = kDefaultWaitNs, bool skip_loads = false);
+
+// One DiT self-attention step on packed QKV in page-locked host memory,
+// through caller-owned device buffers of the same shapes; transfers and
+// kernels overlapped chunk by chunk (host_pipeline.cu). Arguments are assumed
+// validated by the ABI layer.
+struct HostStep {
+  const void* qkv_host;
+  void* out_host;
+  void* qkv_dev;
+  void* out_dev;
+  int64_t batch, S;
+  int32_t F, H, W, heads, heads_per_chunk;
+  const void* gamma_q;
+  const void* gamma_k;
+  float eps, theta, scale;
+};
+cudaError_t enqueue_dit_attn_host(const HostStep& step, cudaStream_t stream);
 
 // Synchronise the stream, then read and clear a kernel's device error word.
 cudaError_t read_and_clear_device_error(cudaStream_t stream, int32_t* code);

@@ -54,6 +54,7 @@ def _load():
             lib.wan_oracle_qk_norm_rope_tokens.argtypes = [P, I64, I32, I32, I32, I32, P, P, D, D,
                                                            P, I64, P]
             lib.wan_oracle_attention_rows.argtypes = [P, I64, I64, I32, D, P, I64, P]
+            lib.wan_oracle_attention_skip_groups.argtypes = [P, I64, I64, I32, D, D, P, I64, P, P, P]
             _lib = lib
     return _lib
 
@@ -143,6 +144,24 @@ def attention_rows(qkv: torch.Tensor, heads: int, rows, scale: float) -> np.ndar
     _load().wan_oracle_attention_rows(_ptr(src), B, S, heads, float(scale), _ptr(r), r.shape[0],
                                       _ptr(out))
     return out
+
+
+def attention_skip_groups(qkv: torch.Tensor, heads: int, groups, scale: float, threshold: float):
+    """Step 4 with Skip-Softmax (threshold mode) for listed (b, h, g) groups of
+    32 query rows: (out fp64 [n, 32, 128] (rows past S: NaN), skipped bool
+    [n, ceil(S/128)], margin fp64 [n]) -- see wan_oracle_attention_skip_groups."""
+    B, S, D3 = qkv.shape
+    assert D3 == 3 * heads * HEAD_DIM
+    g = np.ascontiguousarray(np.asarray(groups, dtype=np.int64).reshape(-1, 3))
+    assert (g[:, 0] < B).all() and (g[:, 1] < heads).all() and (g[:, 2] * 32 < S).all() and (g >= 0).all()
+    n_tiles = (S + 127) // 128
+    out = np.empty((g.shape[0], 32, HEAD_DIM), dtype=np.float64)
+    skipped = np.zeros((g.shape[0], n_tiles), dtype=np.uint8)
+    margin = np.empty(g.shape[0], dtype=np.float64)
+    src = _bits(qkv)
+    _load().wan_oracle_attention_skip_groups(_ptr(src), B, S, heads, float(scale), float(threshold),
+                                             _ptr(g), g.shape[0], _ptr(out), _ptr(skipped), _ptr(margin))
+    return out, skipped.astype(bool), margin
 
 
 def attention_full(qkv: torch.Tensor, heads: int, scale: float) -> np.ndarray:

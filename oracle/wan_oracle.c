@@ -228,3 +228,100 @@ void wan_oracle_attention_rows(const uint16_t* qkv, int64_t batch, int64_t S, in
     }
   }
 }
+
+/* Step 4 with Skip-Softmax in threshold mode (vLLM-Omni "Wan2.2 Text-to-Video"
+ * recipe, "Accelerating with TRTLLM_ATTN + Skip-Softmax": a direct skip
+ * threshold, no calibration). The pages name the threshold but not the rule;
+ * the reading implemented here:
+ *   - keys come in tiles of 128 (tile j = keys [128j, 128j+128) below S);
+ *     query rows in groups of 32 (group g = rows [32g, 32g+32));
+ *   - in base-2 units, a_ik = (q_i . k_k) * scale * log2(e); t_ij is row i's
+ *     largest a_ik over tile j, M_i(j) its largest a_ik over tiles < j;
+ *   - tile j >= 1 is skipped for the group when every row i of the group has
+ *     t_ij < M_i(j) + log2(threshold), i.e. every weight of the tile is below
+ *     `threshold` times the row's running maximum weight. A skipped tile
+ *     contributes neither to the row sum nor to the weighted sum of V. Tile 0
+ *     is never skipped; threshold 0 means dense. A group with a row at or past
+ *     S (a zero query: all its a_ik are 0) never skips.
+ *   - o_i = sum over kept keys of exp(a_ik ln2 - m) v_k / sum of the same
+ *     weights, m the row's largest a over kept keys (fp64, two passes).
+ * groups: n triplets (b, h, g). out: n x 32 x 128 fp64 (rows past S: NaN).
+ * skipped: n x n_tiles bytes (1 = skipped). margin: per group, the smallest
+ * |max_i (t_ij - M_i(j)) - log2(threshold)| over its tiles j >= 1 (+inf when
+ * none), so that a test can tell decisions that rounding could flip. */
+void wan_oracle_attention_skip_groups(const uint16_t* qkv, int64_t batch, int64_t S, int32_t heads,
+                                      double scale, double threshold, const int64_t* groups,
+                                      int64_t n, double* out, uint8_t* skipped, double* margin) {
+  (void)batch;
+  const int64_t D = (int64_t)heads * HEAD_DIM, D3 = 3 * D;
+  const int64_t n_tiles = (S + 127) / 128;
+  const double lg = threshold > 0.0 ? log2(threshold) : -INFINITY;
+  const double to_base2 = scale * 1.4426950408889634074;  /* log2(e) */
+#pragma omp parallel
+  {
+    double* a = (double*)malloc((size_t)(32 * S) * sizeof(double));
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t r = 0; r < n; ++r) {
+      const int64_t b = groups[3 * r], h = groups[3 * r + 1], g = groups[3 * r + 2];
+      const uint16_t* base = qkv + b * S * D3;
+      const int64_t i0 = 32 * g;
+      int has_pad = 0;
+      for (int64_t ii = 0; ii < 32; ++ii) {
+        const int64_t i = i0 + ii;
+        if (i >= S) {
+          has_pad = 1;
+          for (int64_t k = 0; k < S; ++k) a[ii * S + k] = 0.0;
+          continue;
+        }
+        double q[HEAD_DIM];
+        for (int d = 0; d < HEAD_DIM; ++d) q[d] = bf16_to_f64(base[i * D3 + h * HEAD_DIM + d]);
+        for (int64_t k = 0; k < S; ++k) {
+          const uint16_t* kk = base + k * D3 + D + h * HEAD_DIM;
+          double dot = 0.0;
+          for (int d = 0; d < HEAD_DIM; ++d) dot += q[d] * bf16_to_f64(kk[d]);
+          a[ii * S + k] = dot * to_base2;
+        }
+      }
+      /* the decisions */
+      uint8_t* sk = skipped + r * n_tiles;
+      double mg = INFINITY;
+      sk[0] = 0;
+      for (int64_t j = 1; j < n_tiles; ++j) {
+        const int64_t k0 = 128 * j, k1 = (k0 + 128 < S) ? k0 + 128 : S;
+        double worst = -INFINITY; /* max over rows of t_ij - M_i(j) */
+        for (int64_t ii = 0; ii < 32; ++ii) {
+          double M = -INFINITY, t = -INFINITY;
+          for (int64_t k = 0; k < k0; ++k) M = fmax(M, a[ii * S + k]);
+          for (int64_t k = k0; k < k1; ++k) t = fmax(t, a[ii * S + k]);
+          worst = fmax(worst, t - M);
+        }
+        sk[j] = (!has_pad && worst < lg) ? 1 : 0;
+        if (isfinite(lg)) mg = fmin(mg, fabs(worst - lg));
+      }
+      margin[r] = mg;
+      /* the weighted sums over kept tiles */
+      for (int64_t ii = 0; ii < 32; ++ii) {
+        double* o = out + (r * 32 + ii) * HEAD_DIM;
+        if (i0 + ii >= S) {
+          for (int d = 0; d < HEAD_DIM; ++d) o[d] = NAN;
+          continue;
+        }
+        double m = -INFINITY;
+        for (int64_t k = 0; k < S; ++k)
+          if (!sk[k / 128]) m = fmax(m, a[ii * S + k]);
+        double acc[HEAD_DIM];
+        for (int d = 0; d < HEAD_DIM; ++d) acc[d] = 0.0;
+        double sum = 0.0;
+        for (int64_t k = 0; k < S; ++k) {
+          if (sk[k / 128]) continue;
+          const uint16_t* v = base + k * D3 + 2 * D + h * HEAD_DIM;
+          const double w = exp2(a[ii * S + k] - m);
+          sum += w;
+          for (int d = 0; d < HEAD_DIM; ++d) acc[d] += w * bf16_to_f64(v[d]);
+        }
+        for (int d = 0; d < HEAD_DIM; ++d) o[d] = acc[d] / sum;
+      }
+    }
+    free(a);
+  }
+}

@@ -126,6 +126,35 @@ WAN_API int32_t wan_self_attention(const void* qkv, void* out, int64_t batch, in
                            int32_t heads, int32_t head_dim, float scale, void* stream);
 
 /*
+ * (2) with Skip-Softmax in threshold mode (vLLM-Omni "Wan2.2 Text-to-Video"
+ * recipe, "Accelerating with TRTLLM_ATTN + Skip-Softmax": a direct skip
+ * threshold, no calibration; the output diverges from dense as the
+ * threshold grows). Rule, per query tile of 128 rows and key tile j >= 1 of
+ * 128 keys, in groups of 32 query rows: a group skips key tile j when each of
+ * its rows has every weight of the tile below threshold x the row's largest
+ * weight over key tiles 0..j-1 (in scores: tile max < running max +
+ * ln(threshold)). A skipped tile adds nothing to the group's row sums and
+ * weighted sums; when all four groups of a query tile skip, the P V product
+ * is not run. Tile 0 is never skipped; a group holding rows past seq_len
+ * never skips. threshold == 0 runs the dense kernel (bit-identical to
+ * wan_self_attention); threshold must be finite and >= 0.
+ * Other arguments as for wan_self_attention. Counters of what was skipped:
+ * wan_skip_stats.
+ */
+WAN_API int32_t wan_self_attention_sparse(const void* qkv, void* out, int64_t batch, int64_t seq_len,
+                                          int32_t heads, int32_t head_dim, float scale, float threshold,
+                                          void* stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the Skip-Softmax counters
+ * accumulated by wan_self_attention_sparse launches since the last read:
+ * *group_tiles = (32-row group, key tile) pairs skipped, *products = 128-row
+ * P V products skipped. Either pointer may be NULL. Returns WAN_ERR_LAUNCH
+ * when the synchronisation reports a CUDA error.
+ */
+WAN_API int32_t wan_skip_stats(void* stream, int64_t* group_tiles, int64_t* products);
+
+/*
  * (1) then (2) on one stream, the second launch chained to the first with
  * programmatic dependent launch so its prologue overlaps the first's tail.
  * Same arguments and in-place semantics as the two calls above, with

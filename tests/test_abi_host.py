@@ -39,7 +39,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings(lib):
-    assert lib.wan_abi_version() == 3
+    assert lib.wan_abi_version() == 4
     for code in range(11):
         assert lib.wan_status_string(code)
     assert lib.wan_status_string(99) == b"unknown status"
@@ -131,3 +131,11 @@ def test_host_pipeline_validates_before_touching_memory(lib):
     import torch
     if not torch.cuda.is_available():
         assert call() == 6  # valid arguments, no B200: fails loudly
+
+
+def test_sparse_attention_validates_threshold(lib):
+    # (qkv, out, batch, seq_len, heads, head_dim, scale, threshold)
+    assert lib.wan_self_attention_sparse(FAKE, FAKE * 16, 1, 8, 1, 128, 0.0, -0.1, None) == 5
+    assert lib.wan_self_attention_sparse(FAKE, FAKE * 16, 1, 8, 1, 128, 0.0, float("nan"), None) == 5
+    assert lib.wan_self_attention_sparse(FAKE, FAKE * 16, 1, 8, 1, 127, 0.0, 0.1, None) == 4
+    assert lib.wan_self_attention_sparse(FAKE, FAKE + 64, 1, 8, 1, 128, 0.0, 0.1, None) == 9

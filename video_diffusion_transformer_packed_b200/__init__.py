@@ -19,7 +19,7 @@ import threading
 from typing import Optional, Sequence
 
 __all__ = ["WanError", "load_library", "library_path", "qk_norm_rope", "self_attention",
-           "dit_attn", "dit_attn_host", "device_error", "selftest_wait_timeout", "HEAD_DIM", "EPS",
+           "self_attention_sparse", "skip_stats", "dit_attn", "dit_attn_host", "device_error", "selftest_wait_timeout", "HEAD_DIM", "EPS",
            "THETA", "STATUS"]
 
 HEAD_DIM = 128
@@ -76,6 +76,10 @@ def load_library() -> ctypes.CDLL:
             lib.wan_dit_attn_host.argtypes = [P, P, P, P, I64, I32, I32, I32, I32, I32, P, P, F, F, F,
                                               I32, P]
             lib.wan_dit_attn_host.restype = I32
+            lib.wan_self_attention_sparse.argtypes = [P, P, I64, I64, I32, I32, F, F, P]
+            lib.wan_self_attention_sparse.restype = I32
+            lib.wan_skip_stats.argtypes = [P, ctypes.POINTER(I64), ctypes.POINTER(I64)]
+            lib.wan_skip_stats.restype = I32
             _lib = lib
     return _lib
 
@@ -146,6 +150,27 @@ def self_attention(qkv, heads: int, out=None, scale: float = 0.0, stream=None):
                                              heads, HEAD_DIM, scale, _stream(stream)),
            "wan_self_attention")
     return out
+
+
+def self_attention_sparse(qkv, heads: int, threshold: float, out=None, scale: float = 0.0, stream=None):
+    """Softmax attention with Skip-Softmax in threshold mode (0 = dense)."""
+    import torch
+    _check_packed(qkv, heads)
+    B, S, _ = qkv.shape
+    if out is None:
+        out = torch.empty((B, S, heads * HEAD_DIM), dtype=torch.bfloat16, device=qkv.device)
+    _check_out(out, qkv, heads)
+    _check(load_library().wan_self_attention_sparse(_bf16_cuda(qkv, "qkv"), _bf16_cuda(out, "out"), B, S,
+                                                    heads, HEAD_DIM, scale, float(threshold),
+                                                    _stream(stream)), "wan_self_attention_sparse")
+    return out
+
+
+def skip_stats(stream=None):
+    """Synchronise; return and clear (group-tiles skipped, P V products skipped)."""
+    g, p = ctypes.c_int64(0), ctypes.c_int64(0)
+    _check(load_library().wan_skip_stats(_stream(stream), ctypes.byref(g), ctypes.byref(p)), "wan_skip_stats")
+    return g.value, p.value
 
 
 def dit_attn(qkv, grid: Sequence[int], heads: int, gamma_q, gamma_k, out=None, eps: float = EPS,

@@ -11,7 +11,7 @@
 
 namespace {
 
-constexpr int32_t kAbiVersion = 3;
+constexpr int32_t kAbiVersion = 4;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -163,6 +163,36 @@ int32_t wan_self_attention(const void* qkv, void* out, int64_t batch, int64_t se
   if (wan::launch_attn_fwd(plan, static_cast<cudaStream_t>(stream), false) != cudaSuccess) {
     return WAN_ERR_LAUNCH;
   }
+  return WAN_OK;
+}
+
+int32_t wan_self_attention_sparse(const void* qkv, void* out, int64_t batch, int64_t seq_len,
+                                  int32_t heads, int32_t head_dim, float scale, float threshold,
+                                  void* stream) {
+  WAN_TRY(check_heads(heads, head_dim));
+  WAN_TRY(check_tokens(batch, seq_len, heads));
+  WAN_TRY(check_attn_args(qkv, out, batch, seq_len, heads, scale));
+  if (!(std::isfinite(threshold) && threshold >= 0.f)) return WAN_ERR_PARAM;
+  WAN_TRY(check_device());
+  (void)cudaGetLastError();
+  wan::AttnPlan plan;
+  if (wan::plan_attn_fwd(qkv, out, batch, seq_len, heads, scale, &plan) != cudaSuccess) {
+    return WAN_ERR_LAUNCH;
+  }
+  plan.skip_threshold = threshold;
+  if (wan::launch_attn_fwd(plan, static_cast<cudaStream_t>(stream), false) != cudaSuccess) {
+    return WAN_ERR_LAUNCH;
+  }
+  return WAN_OK;
+}
+
+int32_t wan_skip_stats(void* stream, int64_t* group_tiles, int64_t* products) {
+  int64_t g = 0, pr = 0;
+  if (wan::read_and_clear_skip_stats(static_cast<cudaStream_t>(stream), &g, &pr) != cudaSuccess) {
+    return WAN_ERR_LAUNCH;
+  }
+  if (group_tiles) *group_tiles = g;
+  if (products) *products = pr;
   return WAN_OK;
 }
 

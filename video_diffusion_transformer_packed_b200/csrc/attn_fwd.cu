@@ -65,6 +65,7 @@ static_assert(128 * kCtlRegs + 256 * kSoftmaxRegs <= kThreads * kLaunchRegs, "re
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait (the default limit)
 constexpr float kRescaleThreshold = 8.0f;         // log2 of the largest tolerated growth
+constexpr uint32_t kAllGroupsSkipped = 0x01010101u;  // Skip-Softmax votes of the four warps
 // P_t is handed to the MMA issuer in kPParts column blocks, each with its own
 // barrier: O_t += P_t V starts on the first keys while the softmax is still
 // exponentiating the last ones.
@@ -77,13 +78,16 @@ constexpr int kOffQ = 0;                              // 2 tiles
 constexpr int kOffKV = kOffQ + 2 * kTileBytes;        // kStages tiles
 constexpr int kOffBar = kOffKV + kStages * kTileBytes;
 constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 * kPParts + 2 + 1;  // q, kv full/empty, s, p, o, drain
-constexpr int kOffMisc = kOffBar + kNumBars * 8;
+constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tmem holder, abort flag, issued[], votes[8]
 constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + alignment slack
 
 // Error-word site codes.
 constexpr int kErrProducer = 1, kErrMma = 2, kErrSoftmax = 4, kErrEpilogue = 8, kErrDrain = 16;
 
 __device__ int g_attn_error_word;
+// Skip-Softmax counters: [0] (32-row group, key tile) pairs skipped, [1] P V
+// products skipped (all four groups of a query tile skipped the key tile).
+__device__ unsigned long long g_attn_skip_stats[2];
 
 struct AttnParams {
   uint16_t* out;
@@ -93,6 +97,7 @@ struct AttnParams {
   int32_t q_pairs;  // ceil(S / 256): CTAs per (batch, head)
   int32_t n_kv;     // ceil(S / 128)
   int32_t b0, h0, nh;  // this launch covers batches [b0, ...) and heads [h0, h0 + nh)
+  float skip_log2;     // Skip-Softmax: log2 of the threshold (used by the kSkip kernel only)
   float scale_log2; // scale * log2(e)
   uint64_t wait_ns; // limit of each pipeline wait
   int32_t skip_loads;  // self-test: the producer starts no copies, so the waits run out
@@ -167,8 +172,9 @@ __device__ void drain_producer(Bars bars, const int* issued) {
 }
 
 // -------------------------------------------------------------- MMA issuer
+template <bool kSkip>
 __device__ void run_mma(const AttnParams& p, uint32_t smem, Bars bars, volatile int* abort,
-                        uint32_t tmem) {
+                        uint32_t tmem, const volatile uint32_t* votes) {
   constexpr uint32_t kIdescQK = idesc_bf16_f32(kBM, kBN, 0);
   constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, kHD, 1);
   // Descriptors are built once; a step only adds a byte offset (in 16-byte
@@ -219,6 +225,7 @@ __device__ void run_mma(const AttnParams& p, uint32_t smem, Bars bars, volatile 
 
   bool ok = mbar_wait(bars.q_full(), 0, abort, p.wait_ns) && mbar_wait(kv_bar(0), 0, abort, p.wait_ns);
   bool next_v = false, next_p = false;  // probes of V_j and P_0(j) part 0
+  uint32_t n_pv_skipped = 0;
   if (ok) {
     tc_fence_after();
     qk_steps(0, 0, 0, 8);
@@ -242,14 +249,25 @@ __device__ void run_mma(const AttnParams& p, uint32_t smem, Bars bars, volatile 
     }
     // O_0 += P_0 V_j, one block of P at a time.
     bool probe = false;
+    if (kSkip && votes[0] == kAllGroupsSkipped) {
+      // Every warp of query tile 0 skipped key tile j: no product. The other
+      // blocks' arrivals are still awaited, so that the warps' stores of
+      // P = 0 are done before S_0 is rewritten.
 #pragma unroll
-    for (int part = 0; part < kPParts; ++part) {
-      if (part > 0 && !ensure(probe, bars.p_full(0, part), pj)) { ok = false; break; }
-      const int k0 = part * kStepsPerPart, k1 = k0 + kStepsPerPart;
-      pv_steps(0, sv, k0, k1 - 1, acc);
-      probe = part + 1 < kPParts ? mbar_test(bars.p_full(0, part + 1), pj)
-                                 : (more ? mbar_test(kv_bar(ik), kv_par(ik)) : true);
-      pv_steps(0, sv, k1 - 1, k1, acc);
+      for (int part = 1; part < kPParts; ++part) {
+        if (!ensure(false, bars.p_full(0, part), pj)) { ok = false; break; }
+      }
+      ++n_pv_skipped;
+    } else {
+#pragma unroll
+      for (int part = 0; part < kPParts; ++part) {
+        if (part > 0 && !ensure(probe, bars.p_full(0, part), pj)) { ok = false; break; }
+        const int k0 = part * kStepsPerPart, k1 = k0 + kStepsPerPart;
+        pv_steps(0, sv, k0, k1 - 1, acc);
+        probe = part + 1 < kPParts ? mbar_test(bars.p_full(0, part + 1), pj)
+                                   : (more ? mbar_test(kv_bar(ik), kv_par(ik)) : true);
+        pv_steps(0, sv, k1 - 1, k1, acc);
+      }
     }
     if (!ok) break;
     if (more) {
@@ -263,13 +281,22 @@ __device__ void run_mma(const AttnParams& p, uint32_t smem, Bars bars, volatile 
       probe = mbar_test(bars.p_full(1, 0), pj);
     }
     // O_1 += P_1 V_j
+    if (!ensure(probe, bars.p_full(1, 0), pj)) { ok = false; break; }
+    if (kSkip && votes[1] == kAllGroupsSkipped) {
 #pragma unroll
-    for (int part = 0; part < kPParts; ++part) {
-      if (!ensure(probe, bars.p_full(1, part), pj)) { ok = false; break; }
-      const int k0 = part * kStepsPerPart, k1 = k0 + kStepsPerPart;
-      pv_steps(1, sv, k0, k1 - 1, acc);
-      probe = part + 1 < kPParts ? mbar_test(bars.p_full(1, part + 1), pj) : false;
-      pv_steps(1, sv, k1 - 1, k1, acc);
+      for (int part = 1; part < kPParts; ++part) {
+        if (!ensure(false, bars.p_full(1, part), pj)) { ok = false; break; }
+      }
+      ++n_pv_skipped;
+    } else {
+#pragma unroll
+      for (int part = 0; part < kPParts; ++part) {
+        if (part > 0 && !ensure(probe, bars.p_full(1, part), pj)) { ok = false; break; }
+        const int k0 = part * kStepsPerPart, k1 = k0 + kStepsPerPart;
+        pv_steps(1, sv, k0, k1 - 1, acc);
+        probe = part + 1 < kPParts ? mbar_test(bars.p_full(1, part + 1), pj) : false;
+        pv_steps(1, sv, k1 - 1, k1, acc);
+      }
     }
     if (!ok) break;
     mma_commit(bars.kv_empty(sv));
@@ -283,6 +310,7 @@ __device__ void run_mma(const AttnParams& p, uint32_t smem, Bars bars, volatile 
       mma_commit(bars.kv_empty(sk));
     }
   }
+  if (kSkip && n_pv_skipped) atomicAdd(&g_attn_skip_stats[1], n_pv_skipped);
   if (ok) {
     mma_commit(bars.o_full(0));
     mma_commit(bars.o_full(1));
@@ -295,14 +323,19 @@ __device__ void run_mma(const AttnParams& p, uint32_t smem, Bars bars, volatile 
 }
 
 // ----------------------------------------------------------------- softmax
+template <bool kSkip>
 __device__ void run_softmax(const AttnParams& p, Bars bars, volatile int* abort, uint32_t tmem,
-                            int t, int quarter, int lane, int b, int h, int qp) {
+                            int t, int quarter, int lane, int b, int h, int qp,
+                            volatile uint8_t* votes) {
   const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
   const uint32_t tS = tmem + lane_base + t * 128;
   const uint32_t tO = tmem + lane_base + 256 + t * 128;
   const float sl2 = p.scale_log2;
   float m_run = -INFINITY;  // running max, already in scaled log2 units
   float l_run = 0.f;
+  float m_true = -INFINITY;  // exact running max (Skip-Softmax decisions)
+  const bool row_valid = (2 * qp + t) * kBM + quarter * 32 + lane < p.S;
+  uint32_t n_skipped = 0;
   bool ok = true;
 
 #pragma unroll 1
@@ -333,6 +366,31 @@ __device__ void run_softmax(const AttnParams& p, Bars bars, volatile int* abort,
     }
     const float mx = fmaxf(max3(mk[0], mk[1], mk[2]), max3(max3(mk[3], mk[4], mk[5]), mk[6], mk[7]));
     const float m_cand = mx * sl2;
+    if constexpr (kSkip) {
+      // Skip-Softmax, threshold mode: the warp's 32 rows skip this key tile
+      // when each row's largest weight in it is below threshold x the row's
+      // running maximum weight (a row past S never votes to skip). The rows
+      // get P = 0, since the tile's O += P V still runs when another warp of
+      // the query tile keeps it; the MMA issuer drops the product when all
+      // four warps skip.
+      const bool row_skip = row_valid && m_cand < m_true + p.skip_log2;
+      m_true = fmaxf(m_true, m_cand);
+      const bool warp_skip = __all_sync(0xffffffffu, row_skip);
+      if (lane == 0) votes[t * 4 + quarter] = warp_skip ? 1 : 0;
+      if (warp_skip) {
+        uint32_t z[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) z[e] = 0u;
+        tmem_st32(tS, z);
+        tmem_st32(tS + 32, z);
+        tmem_wait_st();
+        tc_fence_before();
+#pragma unroll
+        for (int part = 0; part < kPParts; ++part) mbar_arrive(bars.p_full(t, part));
+        ++n_skipped;
+        continue;
+      }
+    }
     const bool raise = m_cand > m_run + kRescaleThreshold;
     float alpha = 1.f;
     if (raise) {
@@ -387,6 +445,7 @@ __device__ void run_softmax(const AttnParams& p, Bars bars, volatile int* abort,
     f2_split(add2(add2(sum2[0], sum2[1]), add2(sum2[2], sum2[3])), sum_lo, sum_hi);
     l_run += sum_lo + sum_hi;
   }
+  if (kSkip && lane == 0 && n_skipped) atomicAdd(&g_attn_skip_stats[0], n_skipped);
   if (!ok) {
     flag_error(abort, kErrSoftmax);
     return;
@@ -416,6 +475,7 @@ __device__ void run_softmax(const AttnParams& p, Bars bars, volatile int* abort,
   }
 }
 
+template <bool kSkip>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -426,6 +486,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
   int* issued = reinterpret_cast<int*>(smem + kOffMisc + 8);  // [kStages + 1], producer-owned
+  // Skip-Softmax votes: byte [t * 4 + w] = warp w of query tile t skipped the current key tile.
+  uint8_t* votes = smem + kOffMisc + 32;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -448,6 +510,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bars.drain(), 1);
     *abort = 0;
     for (int s = 0; s <= kStages; ++s) issued[s] = 0;
+    for (int v = 0; v < 8; ++v) votes[v] = 0;
     fence_mbar_init();
   }
   if (warp == kMmaWarp) {
@@ -465,12 +528,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kLoadWarp) {
       if (lane == 0) run_producer(&tmap, p, smem_base, bars, abort, issued, b, h, qp);
     } else if (warp == kMmaWarp) {
-      if (lane == 0) run_mma(p, smem_base, bars, abort, tmem);
+      if (lane == 0) {
+        run_mma<kSkip>(p, smem_base, bars, abort, tmem, reinterpret_cast<const volatile uint32_t*>(votes));
+      }
     }
     __syncwarp();
   } else {
     regs_increase<kSoftmaxRegs>();
-    run_softmax(p, bars, abort, tmem, warp >> 2, warp & 3, lane, b, h, qp);
+    run_softmax<kSkip>(p, bars, abort, tmem, warp >> 2, warp & 3, lane, b, h, qp, votes);
   }
 
   tc_fence_before();
@@ -512,12 +577,14 @@ cudaError_t plan_attn_fwd(const void* qkv, void* out, int64_t batch, int64_t seq
   std::call_once(attr_once, [] {
     // The register split inside the kernel is only safe when the compiled
     // kernel launches with exactly kLaunchRegs registers per thread.
-    cudaFuncAttributes fa;
-    attr_err = cudaFuncGetAttributes(&fa, attn_fwd_kernel);
-    if (attr_err == cudaSuccess && fa.numRegs != kLaunchRegs) attr_err = cudaErrorInvalidKernelImage;
-    if (attr_err == cudaSuccess) {
-      attr_err = cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      kSmemBytes);
+    for (auto kernel : {attn_fwd_kernel<false>, attn_fwd_kernel<true>}) {
+      cudaFuncAttributes fa;
+      attr_err = cudaFuncGetAttributes(&fa, kernel);
+      if (attr_err == cudaSuccess && fa.numRegs != kLaunchRegs) attr_err = cudaErrorInvalidKernelImage;
+      if (attr_err == cudaSuccess) {
+        attr_err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+      }
+      if (attr_err != cudaSuccess) return;
     }
   });
   if (attr_err != cudaSuccess) return attr_err;
@@ -544,6 +611,7 @@ cudaError_t plan_attn_fwd(const void* qkv, void* out, int64_t batch, int64_t seq
   plan->n_kv = (S + kBN - 1) / kBN;
   const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(kHD));
   plan->scale_log2 = sc * 1.4426950408889634f;
+  plan->skip_threshold = 0.f;
   plan->b0 = 0;
   plan->nb = static_cast<int32_t>(batch);
   plan->h0 = 0;
@@ -564,6 +632,7 @@ cudaError_t launch_attn_fwd(const AttnPlan& plan, cudaStream_t stream, bool pdl,
   p.h0 = plan.h0;
   p.nh = plan.nh;
   p.scale_log2 = plan.scale_log2;
+  p.skip_log2 = plan.skip_threshold > 0.f ? log2f(plan.skip_threshold) : -INFINITY;
   p.wait_ns = wait_ns;
   p.skip_loads = skip_loads ? 1 : 0;
   CUtensorMap tmap;
@@ -584,7 +653,22 @@ cudaError_t launch_attn_fwd(const AttnPlan& plan, cudaStream_t stream, bool pdl,
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, attn_fwd_kernel, tmap, p);
+  if (plan.skip_threshold > 0.f) return cudaLaunchKernelEx(&cfg, attn_fwd_kernel<true>, tmap, p);
+  return cudaLaunchKernelEx(&cfg, attn_fwd_kernel<false>, tmap, p);
+}
+
+cudaError_t read_and_clear_skip_stats(cudaStream_t stream, int64_t* group_tiles, int64_t* products) {
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return e;
+  unsigned long long v[2] = {0, 0};
+  e = cudaMemcpyFromSymbol(v, g_attn_skip_stats, sizeof(v));
+  if (e != cudaSuccess) return e;
+  const unsigned long long zero[2] = {0, 0};
+  e = cudaMemcpyToSymbol(g_attn_skip_stats, zero, sizeof(zero));
+  if (e != cudaSuccess) return e;
+  *group_tiles = static_cast<int64_t>(v[0]);
+  *products = static_cast<int64_t>(v[1]);
+  return cudaSuccess;
 }
 
 cudaError_t read_and_clear_device_error(cudaStream_t stream, int32_t* code) {

@@ -25,6 +25,8 @@ struct AttnPlan {
   // [h0, h0 + nh). plan_attn_fwd sets the whole buffer; a pipelined caller
   // narrows a copy of the plan per launch.
   int32_t b0, nb, h0, nh;
+  // Skip-Softmax threshold (0 = dense; plan_attn_fwd sets 0).
+  float skip_threshold;
 };
 
 cudaError_t plan_attn_fwd(const void* qkv, void* out, int64_t batch, int64_t seq_len,
@@ -54,6 +56,10 @@ struct HostStep {
   float eps, theta, scale;
 };
 cudaError_t enqueue_dit_attn_host(const HostStep& step, cudaStream_t stream);
+
+// Synchronise the stream, then read and clear the Skip-Softmax counters:
+// (32-row group, key tile) pairs skipped, and P V products skipped.
+cudaError_t read_and_clear_skip_stats(cudaStream_t stream, int64_t* group_tiles, int64_t* products);
 
 // Synchronise the stream, then read and clear a kernel's device error word.
 cudaError_t read_and_clear_device_error(cudaStream_t stream, int32_t* code);

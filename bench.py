@@ -56,6 +56,7 @@ def parse_args():
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-skip", action="store_true", help="skip the Skip-Softmax side measurement")
     return ap.parse_args()
 
 
@@ -352,6 +353,39 @@ def run_ours(args):
                "h2d_bytes_per_step": qkv.numel() * 2, "d2h_bytes_per_step": out.numel() * 2,
                "ms_per_step": e2e_ms / args.steps}
 
+    # ---- Skip-Softmax side measurement (not the headline): same shape, inputs
+    # with local, peaked attention (wan_inputs.local_peaked_qkv), dense kernel
+    # vs threshold mode, device time of one launch each, skipped fractions
+    # from the kernel's own counters.
+    skip = None
+    if not args.no_skip:
+        loc = wi.local_peaked_qkv(w.batch, w.seq_len, w.heads, seed=5).to(dev)
+        n_t = (w.seq_len + 127) // 128
+        reps = 3
+
+        def timed(thr):
+            with torch.cuda.stream(stream):
+                wan.self_attention_sparse(loc, w.heads, thr, out=out, stream=stream)
+            wan.skip_stats(stream)
+            a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(reps):
+                wan.self_attention_sparse(loc, w.heads, thr, out=out, stream=stream)
+            b_.record(stream)
+            b_.synchronize()
+            tiles, prods = wan.skip_stats(stream)
+            return a.elapsed_time(b_) / reps, tiles / reps, prods / reps
+
+        dense_ms, _, _ = timed(0.0)
+        skip = {"workload": "local peaked synthetic (each query alpha=0.6 times a key within 8 tokens), "
+                            + w.name, "dense_ms": dense_ms, "points": []}
+        for thr in (0.02, 0.05):
+            ms_, tiles, prods = timed(thr)
+            skip["points"].append({"threshold": thr, "ms": ms_, "speedup_vs_dense": dense_ms / ms_,
+                                   "group_tiles_skipped": tiles / (w.batch * w.heads * 4 * n_t * n_t),
+                                   "products_skipped": prods / (w.batch * w.heads * n_t * n_t)})
+        del loc
+
     peaks, peak_src = load_peaks()
     tensor_peak = peaks["bf16_tflops_sustained"]
     roofline = {
@@ -393,7 +427,7 @@ def run_ours(args):
         "attn_tflops": attn_tflops, "attn_frac_of_peak": attn_tflops / tensor_peak,
         "norm_rope_gbs": norm_gbs, "norm_rope_frac_of_hbm": norm_gbs / peaks["hbm_gbs"],
         "roofline": roofline, "roofline_norm_rope": norm_roofline,
-        "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
+        "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks, "skip_softmax": skip,
         "gpu_launches": 2 * args.steps,
     }
     print(json.dumps(line), flush=True)

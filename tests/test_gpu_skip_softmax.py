@@ -11,6 +11,7 @@ import pytest
 import torch
 
 import oracle
+import wan_inputs as wi
 import video_diffusion_transformer_packed_b200 as wan
 from video_diffusion_transformer_packed_b200 import build as wan_build
 from helpers import assert_attention_close
@@ -27,16 +28,7 @@ def _built():
 
 
 def local_qkv(batch, S, heads, seed, alpha=0.6, reach=8):
-    """N(0,1) keys and values; each query is alpha times a key within `reach`
-    positions of it, so that attention is peaked and local and whole groups of
-    32 rows agree on which distant key tiles hardly matter."""
-    g = torch.Generator().manual_seed(seed)
-    qkv = torch.randn(batch, S, 3 * heads * HD, generator=g)
-    D = heads * HD
-    for b in range(batch):
-        src = (torch.arange(S) + torch.randint(-reach, reach + 1, (S,), generator=g)).clamp(0, S - 1)
-        qkv[b, :, :D] = alpha * qkv[b, src, D:2 * D]
-    return qkv.to(torch.bfloat16)
+    return wi.local_peaked_qkv(batch, S, heads, seed, alpha, reach)
 
 
 def oracle_groups(qkv, heads, threshold):

@@ -98,6 +98,25 @@ def packed_qkv(batch: int, seq_len: int, heads: int, seed: int = 0,
     return out
 
 
+def local_peaked_qkv(batch: int, seq_len: int, heads: int, seed: int = 0, alpha: float = 0.6,
+                     reach: int = 8) -> torch.Tensor:
+    """Packed [B, S, 3*heads*128] bf16 whose attention is local and peaked: K and
+    V ~ N(0,1) as in packed_qkv, and the query of token i is alpha times the key
+    of a token drawn uniformly within `reach` positions of i (clamped to the
+    sequence). A stand-in for the concentrated attention maps that make
+    Skip-Softmax pay off on real activations, which are not available here.
+    """
+    out = packed_qkv(batch, seq_len, heads, seed)
+    D = heads * HEAD_DIM
+    g = torch.Generator().manual_seed(seed + 7919)
+    for b in range(batch):
+        src = (torch.arange(seq_len) + torch.randint(-reach, reach + 1, (seq_len,), generator=g)).clamp(0, seq_len - 1)
+        for r0 in range(0, seq_len, 4096):
+            r1 = min(r0 + 4096, seq_len)
+            out[b, r0:r1, :D] = (alpha * out[b, src[r0:r1], D:2 * D].float()).to(torch.bfloat16)
+    return out
+
+
 def gammas(heads: int, seed_q: int = 1, seed_k: int = 2) -> Tuple[torch.Tensor, torch.Tensor]:
     """RMSNorm weights for Q and K over the full hidden dim, bf16 ~ U(0.5, 1.5)."""
     d = heads * HEAD_DIM

@@ -55,6 +55,12 @@ def _load():
                                                            P, I64, P]
             lib.wan_oracle_attention_rows.argtypes = [P, I64, I64, I32, D, P, I64, P]
             lib.wan_oracle_attention_skip_groups.argtypes = [P, I64, I64, I32, D, D, P, I64, P, P, P]
+            lib.wan_oracle_e4m3_encode.argtypes = [D]
+            lib.wan_oracle_e4m3_encode.restype = ctypes.c_uint8
+            lib.wan_oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+            lib.wan_oracle_e4m3_decode.restype = D
+            lib.wan_oracle_quantize_e4m3.argtypes = [P, I64, ctypes.c_float, P]
+            lib.wan_oracle_attention_fp8_rows.argtypes = [P, P, I64, I64, I64, I32, D, D, D, D, P, I64, P]
             _lib = lib
     return _lib
 
@@ -162,6 +168,51 @@ def attention_skip_groups(qkv: torch.Tensor, heads: int, groups, scale: float, t
     _load().wan_oracle_attention_skip_groups(_ptr(src), B, S, heads, float(scale), float(threshold),
                                              _ptr(g), g.shape[0], _ptr(out), _ptr(skipped), _ptr(margin))
     return out, skipped.astype(bool), margin
+
+
+def e4m3_encode(v: float) -> int:
+    """e4m3 code of a finite value (round to nearest even, saturating at +-448)."""
+    return int(_load().wan_oracle_e4m3_encode(float(v)))
+
+
+def e4m3_decode(c: int) -> float:
+    return float(_load().wan_oracle_e4m3_decode(int(c)))
+
+
+def quantize_e4m3(x: torch.Tensor, inv_scale: float) -> np.ndarray:
+    """Codes (uint8, same shape) of a bf16 tensor: e4m3(fl32(x * inv_scale))."""
+    assert x.dtype == torch.bfloat16
+    src = np.ascontiguousarray(x.contiguous().view(torch.int16).numpy().view(np.uint16))
+    out = np.empty(src.shape, dtype=np.uint8)
+    _load().wan_oracle_quantize_e4m3(_ptr(src), src.size, float(np.float32(inv_scale)), _ptr(out))
+    return out
+
+
+def fp8_operands(qkv: torch.Tensor, heads: int, inv_sq: float, inv_sk: float, inv_sv: float, s_pitch: int):
+    """The e4m3 operands of the FP8 variant from a packed bf16 buffer: qk8
+    [B, S, 2D] (Q then K of each token) and v8t [B, heads, 128, s_pitch] (V
+    transposed, zero codes past S)."""
+    B, S, D3 = qkv.shape
+    D = D3 // 3
+    qk8 = np.concatenate([quantize_e4m3(qkv[..., :D], inv_sq), quantize_e4m3(qkv[..., D:2 * D], inv_sk)], axis=-1)
+    v8 = quantize_e4m3(qkv[..., 2 * D:], inv_sv).reshape(B, S, heads, HEAD_DIM)
+    v8t = np.zeros((B, heads, HEAD_DIM, s_pitch), dtype=np.uint8)
+    v8t[..., :S] = v8.transpose(0, 2, 3, 1)
+    return np.ascontiguousarray(qk8), v8t
+
+
+def attention_fp8_rows(qk8: np.ndarray, v8t: np.ndarray, heads: int, rows, scale: float, sq: float,
+                       sk: float, sv: float) -> np.ndarray:
+    """Step 4 on e4m3 operands (dequantised, fp64) for listed (b, h, i) rows: [n, 128]."""
+    B, S, D2 = qk8.shape
+    assert D2 == 2 * heads * HEAD_DIM and v8t.shape[:3] == (B, heads, HEAD_DIM)
+    r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 3))
+    out = np.empty((r.shape[0], HEAD_DIM), dtype=np.float64)
+    qk8 = np.ascontiguousarray(qk8)
+    v8t = np.ascontiguousarray(v8t)
+    _load().wan_oracle_attention_fp8_rows(_ptr(qk8), _ptr(v8t), B, S, v8t.shape[3], heads, float(scale),
+                                          float(sq), float(sk), float(sv), _ptr(r), r.shape[0], _ptr(out))
+    return out
 
 
 def attention_full(qkv: torch.Tensor, heads: int, scale: float) -> np.ndarray:

@@ -325,3 +325,94 @@ void wan_oracle_attention_skip_groups(const uint16_t* qkv, int64_t batch, int64_
     free(a);
   }
 }
+
+/* ---- FP8 (e4m3) attention variant ------------------------------------------
+ * The path the pages time is FP8 attention (Neuron "Optimizing High-Quality
+ * Offline Video Generation" and the TensorRT-LLM PR's profiling of TE FP8
+ * attention) with per-tensor scales. Reading: a tensor X with scale s is
+ * stored as codes c = e4m3(fl32(x * (1/s))) -- the product rounded to fp32
+ * (the precision the kernel decides the code in), then round to nearest even
+ * onto the e4m3 grid (3 mantissa bits, exponent bias 7, subnormals down to
+ * 2^-9), saturating at +-448 -- and stands for c * s. Attention then runs on
+ * the dequantised Q, K and V (fp64 here). */
+
+/* e4m3 code (sign bit 7) of a finite double, round to nearest even, saturating. */
+uint8_t wan_oracle_e4m3_encode(double v) {
+  const uint8_t sign = (v < 0.0 || (v == 0.0 && signbit(v))) ? 0x80 : 0x00;
+  double a = fabs(v);
+  if (a == 0.0) return sign;
+  int e;
+  (void)frexp(a, &e); /* a = f * 2^e, f in [0.5, 1): the binade's exponent is e - 1 */
+  int eb = e - 1;
+  if (eb < -6) eb = -6; /* below 2^-6 the grid is the subnormal one, step 2^-9 */
+  const double q = ldexp(1.0, eb - 3);
+  double r = nearbyint(a / q) * q; /* exact: a / q is a power-of-two scaling */
+  if (r > 448.0) r = 448.0;
+  if (r == 0.0) return sign;
+  int er;
+  (void)frexp(r, &er);
+  er -= 1;
+  if (er < -6) return (uint8_t)(sign | (uint8_t)(r / ldexp(1.0, -9))); /* subnormal: m * 2^-9 */
+  const int mant = (int)((r / ldexp(1.0, er) - 1.0) * 8.0);
+  return (uint8_t)(sign | (uint8_t)((er + 7) << 3) | (uint8_t)mant);
+}
+
+double wan_oracle_e4m3_decode(uint8_t c) {
+  const double s = (c & 0x80) ? -1.0 : 1.0;
+  const int ef = (c >> 3) & 0xF, m = c & 7;
+  if (ef == 0xF && m == 7) return NAN;
+  if (ef == 0) return s * ldexp((double)m, -9);
+  return s * ldexp(1.0 + m / 8.0, ef - 7);
+}
+
+/* codes of n bf16 values: e4m3(fl32(x * inv_scale)). */
+void wan_oracle_quantize_e4m3(const uint16_t* x, int64_t n, float inv_scale, uint8_t* out) {
+#pragma omp parallel for schedule(static)
+  for (int64_t i = 0; i < n; ++i) {
+    const float xf = (float)bf16_to_f64(x[i]);
+    const float prod = xf * inv_scale; /* one fp32 rounding (contraction is off) */
+    out[i] = wan_oracle_e4m3_encode((double)prod);
+  }
+}
+
+/* Step 4 on e4m3 codes. qk8: [B, S, 2, heads, 128] codes of Q then K;
+ * v8t: [B, heads, 128, s_pitch] codes of V transposed (dimension-major);
+ * sq, sk, sv: the tensors' scales. rows: n triplets (b, h, i). out: n x 128
+ * fp64, the attention of the dequantised values (unrounded). */
+void wan_oracle_attention_fp8_rows(const uint8_t* qk8, const uint8_t* v8t, int64_t batch, int64_t S,
+                                   int64_t s_pitch, int32_t heads, double scale, double sq, double sk,
+                                   double sv, const int64_t* rows, int64_t n, double* out) {
+  (void)batch;
+  const int64_t D = (int64_t)heads * HEAD_DIM, D2 = 2 * D;
+#pragma omp parallel
+  {
+    double* w = (double*)malloc((size_t)S * sizeof(double));
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t r = 0; r < n; ++r) {
+      const int64_t b = rows[3 * r], h = rows[3 * r + 1], i = rows[3 * r + 2];
+      const uint8_t* base = qk8 + b * S * D2;
+      double q[HEAD_DIM];
+      for (int d = 0; d < HEAD_DIM; ++d) q[d] = wan_oracle_e4m3_decode(base[i * D2 + h * HEAD_DIM + d]) * sq;
+      double m = -INFINITY;
+      for (int64_t j = 0; j < S; ++j) {
+        const uint8_t* k = base + j * D2 + D + h * HEAD_DIM;
+        double dot = 0.0;
+        for (int d = 0; d < HEAD_DIM; ++d) dot += q[d] * (wan_oracle_e4m3_decode(k[d]) * sk);
+        w[j] = dot * scale;
+        if (w[j] > m) m = w[j];
+      }
+      double sum = 0.0;
+      for (int64_t j = 0; j < S; ++j) {
+        w[j] = exp(w[j] - m);
+        sum += w[j];
+      }
+      const uint8_t* vt = v8t + (b * heads + h) * (int64_t)HEAD_DIM * s_pitch;
+      for (int d = 0; d < HEAD_DIM; ++d) {
+        double acc = 0.0;
+        for (int64_t j = 0; j < S; ++j) acc += w[j] * (wan_oracle_e4m3_decode(vt[d * s_pitch + j]) * sv);
+        out[r * HEAD_DIM + d] = acc / sum;
+      }
+    }
+    free(w);
+  }
+}

@@ -146,6 +146,38 @@ WAN_API int32_t wan_self_attention_sparse(const void* qkv, void* out, int64_t ba
                                           void* stream);
 
 /*
+ * FP8 (e4m3) variant of (2) -- the attention arithmetic the pages time (Neuron
+ * "Optimizing High-Quality Offline Video Generation"; the TensorRT-LLM PR's TE
+ * FP8 attention profile) -- with per-tensor scales. A tensor X is stored as
+ * codes c = e4m3(fl32(x * inv_scale_X)) (round to nearest even, saturating at
+ * +-448) and stands for c * scale_X; the caller picks the scales (typically
+ * scale_X = amax_X / 448 from wan_qkv_amax, inv_scale_X = 1 / scale_X).
+ *
+ * wan_qkv_amax: max |x| of Q, K and V of the packed bf16 buffer into
+ *   amax[0..2] (device pointer to 3 floats, 4-byte aligned), asynchronously.
+ * wan_quantize_fp8: codes of the packed bf16 buffer:
+ *   qk8  device, [batch][seq_len][2][heads][128] e4m3 (Q then K per token);
+ *   v8t  device, [batch][heads][128][s_pitch] e4m3: V transposed per
+ *        (batch, head), key-contiguous; columns past seq_len hold code 0;
+ *   s_pitch: a multiple of 16, >= seq_len. Both 16-byte aligned.
+ * wan_self_attention_fp8: out[b, i, h, :] = sum_j softmax_j(scale * q_i . k_j) v_j
+ *   on the dequantised operands, both products in kind::f8f6f4 on the tensor
+ *   cores (fp32 accumulation), the probabilities rounded to e4m3 for the P V
+ *   product, out in bf16 [batch][seq_len][heads*128]. scale <= 0 means
+ *   1/sqrt(128). The e4m3 rounding of the operands and of P makes the result
+ *   differ from the bf16 path by a few per cent (relative Frobenius).
+ * Scales finite and > 0; head_dim == 128; buffers must not overlap out.
+ */
+WAN_API int32_t wan_qkv_amax(const void* qkv, int64_t batch, int64_t seq_len, int32_t heads, int32_t head_dim,
+                             float* amax, void* stream);
+WAN_API int32_t wan_quantize_fp8(const void* qkv, void* qk8, void* v8t, int64_t batch, int64_t seq_len,
+                                 int32_t heads, int32_t head_dim, int64_t s_pitch, float inv_scale_q,
+                                 float inv_scale_k, float inv_scale_v, void* stream);
+WAN_API int32_t wan_self_attention_fp8(const void* qk8, const void* v8t, void* out, int64_t batch,
+                                       int64_t seq_len, int32_t heads, int32_t head_dim, int64_t s_pitch,
+                                       float scale, float scale_q, float scale_k, float scale_v, void* stream);
+
+/*
  * Synchronises `stream`, then reads and clears the Skip-Softmax counters
  * accumulated by wan_self_attention_sparse launches since the last read:
  * *group_tiles = (32-row group, key tile) pairs skipped, *products = 128-row
@@ -204,9 +236,11 @@ WAN_API int32_t wan_dit_attn_host(const void* qkv_host, void* out_host, void* qk
                                   void* stream);
 
 /*
- * Synchronises `stream`, then reads and clears the device-side error word
- * that the attention kernel sets when one of its bounded waits gives up.
- * *code receives 0 when no wait gave up, otherwise a nonzero site code.
+ * Synchronises `stream`, then reads and clears the device-side error words
+ * that the kernels set when one of their bounded waits gives up. *code
+ * receives 0 when no wait gave up, otherwise a nonzero value: the bf16
+ * attention's site code in bits 0-7, norm+RoPE's in bits 8-15, the FP8
+ * attention's in bits 16-23.
  * Returns WAN_ERR_DEVICE_TIMEOUT when *code != 0, WAN_ERR_NULL when code is
  * NULL, WAN_ERR_LAUNCH when the synchronisation reports a CUDA error.
  */

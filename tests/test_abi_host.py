@@ -39,7 +39,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings(lib):
-    assert lib.wan_abi_version() == 4
+    assert lib.wan_abi_version() == 5
     for code in range(11):
         assert lib.wan_status_string(code)
     assert lib.wan_status_string(99) == b"unknown status"
@@ -139,3 +139,23 @@ def test_sparse_attention_validates_threshold(lib):
     assert lib.wan_self_attention_sparse(FAKE, FAKE * 16, 1, 8, 1, 128, 0.0, float("nan"), None) == 5
     assert lib.wan_self_attention_sparse(FAKE, FAKE * 16, 1, 8, 1, 127, 0.0, 0.1, None) == 4
     assert lib.wan_self_attention_sparse(FAKE, FAKE + 64, 1, 8, 1, 128, 0.0, 0.1, None) == 9
+
+
+def test_fp8_entry_points_validate(lib):
+    # wan_quantize_fp8(qkv, qk8, v8t, batch, S, heads, head_dim, s_pitch, iq, ik, iv)
+    far1, far2 = 2**40, 2**41
+    assert lib.wan_quantize_fp8(None, far1, far2, 1, 8, 1, 128, 16, 1.0, 1.0, 1.0, None) == 1
+    assert lib.wan_quantize_fp8(FAKE, far1 + 8, far2, 1, 8, 1, 128, 16, 1.0, 1.0, 1.0, None) == 2
+    assert lib.wan_quantize_fp8(FAKE, far1, far2, 1, 20, 1, 128, 16, 1.0, 1.0, 1.0, None) == 3  # pitch < S
+    assert lib.wan_quantize_fp8(FAKE, far1, far2, 1, 8, 1, 128, 24, 1.0, 1.0, 1.0, None) == 3  # pitch % 16
+    assert lib.wan_quantize_fp8(FAKE, far1, far2, 1, 8, 1, 128, 16, 0.0, 1.0, 1.0, None) == 5
+    assert lib.wan_quantize_fp8(FAKE, FAKE + 1024, far2, 1, 8, 1, 128, 16, 1.0, 1.0, 1.0, None) == 9
+    # wan_self_attention_fp8(qk8, v8t, out, batch, S, heads, head_dim, s_pitch, scale, sq, sk, sv)
+    assert lib.wan_self_attention_fp8(far1, far2, FAKE, 1, 8, 1, 64, 16, 0.0, 1.0, 1.0, 1.0, None) == 4
+    assert lib.wan_self_attention_fp8(far1, far2, FAKE, 1, 8, 1, 128, 16, 0.0, -1.0, 1.0, 1.0, None) == 5
+    assert lib.wan_self_attention_fp8(far1, far1 + 64, FAKE, 1, 8, 1, 128, 16, 0.0, 1.0, 1.0, 1.0, None) == 9
+    assert lib.wan_qkv_amax(FAKE, 1, 8, 1, 128, None, None) == 1
+    assert lib.wan_qkv_amax(FAKE, 1, 8, 1, 128, FAKE + 2, None) == 2
+    import torch
+    if not torch.cuda.is_available():
+        assert lib.wan_self_attention_fp8(far1, far2, FAKE, 1, 8, 1, 128, 16, 0.0, 1.0, 1.0, 1.0, None) == 6

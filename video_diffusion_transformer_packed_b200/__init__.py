@@ -19,7 +19,8 @@ import threading
 from typing import Optional, Sequence
 
 __all__ = ["WanError", "load_library", "library_path", "qk_norm_rope", "self_attention",
-           "self_attention_sparse", "skip_stats", "dit_attn", "dit_attn_host", "device_error", "selftest_wait_timeout", "HEAD_DIM", "EPS",
+           "self_attention_sparse", "skip_stats", "qkv_amax", "quantize_fp8", "self_attention_fp8",
+           "fp8_pitch", "dit_attn", "dit_attn_host", "device_error", "selftest_wait_timeout", "HEAD_DIM", "EPS",
            "THETA", "STATUS"]
 
 HEAD_DIM = 128
@@ -80,6 +81,12 @@ def load_library() -> ctypes.CDLL:
             lib.wan_self_attention_sparse.restype = I32
             lib.wan_skip_stats.argtypes = [P, ctypes.POINTER(I64), ctypes.POINTER(I64)]
             lib.wan_skip_stats.restype = I32
+            lib.wan_qkv_amax.argtypes = [P, I64, I64, I32, I32, P, P]
+            lib.wan_qkv_amax.restype = I32
+            lib.wan_quantize_fp8.argtypes = [P, P, P, I64, I64, I32, I32, I64, F, F, F, P]
+            lib.wan_quantize_fp8.restype = I32
+            lib.wan_self_attention_fp8.argtypes = [P, P, P, I64, I64, I32, I32, I64, F, F, F, F, P]
+            lib.wan_self_attention_fp8.restype = I32
             _lib = lib
     return _lib
 
@@ -171,6 +178,69 @@ def skip_stats(stream=None):
     g, p = ctypes.c_int64(0), ctypes.c_int64(0)
     _check(load_library().wan_skip_stats(_stream(stream), ctypes.byref(g), ctypes.byref(p)), "wan_skip_stats")
     return g.value, p.value
+
+
+E4M3_MAX = 448.0
+
+
+def _u8_cuda(t, name: str) -> int:
+    import torch
+    if t.dtype != torch.uint8 or not t.is_cuda or not t.is_contiguous():
+        raise TypeError(f"{name} must be a contiguous uint8 CUDA tensor")
+    return t.data_ptr()
+
+
+def qkv_amax(qkv, heads: int, stream=None):
+    """max |x| of Q, K and V of a packed bf16 buffer: float32 CUDA tensor [3]."""
+    import torch
+    _check_packed(qkv, heads)
+    B, S, _ = qkv.shape
+    amax = torch.empty(3, dtype=torch.float32, device=qkv.device)
+    _check(load_library().wan_qkv_amax(_bf16_cuda(qkv, "qkv"), B, S, heads, HEAD_DIM, amax.data_ptr(),
+                                       _stream(stream)), "wan_qkv_amax")
+    return amax
+
+
+def fp8_pitch(seq_len: int) -> int:
+    return (seq_len + 15) // 16 * 16
+
+
+def quantize_fp8(qkv, heads: int, inv_scales, qk8=None, v8t=None, stream=None):
+    """e4m3 codes of a packed bf16 buffer: (qk8 [B, S, 2*heads*128],
+    v8t [B, heads, 128, s_pitch]) with codes e4m3(fl32(x * inv_scale))."""
+    import torch
+    _check_packed(qkv, heads)
+    B, S, _ = qkv.shape
+    pitch = fp8_pitch(S)
+    if qk8 is None:
+        qk8 = torch.empty((B, S, 2 * heads * HEAD_DIM), dtype=torch.uint8, device=qkv.device)
+    if v8t is None:
+        v8t = torch.empty((B, heads, HEAD_DIM, pitch), dtype=torch.uint8, device=qkv.device)
+    if tuple(qk8.shape) != (B, S, 2 * heads * HEAD_DIM) or v8t.dim() != 4 or tuple(v8t.shape[:3]) != (B, heads, HEAD_DIM):
+        raise ValueError("qk8 must be [B, S, 2*heads*128] and v8t [B, heads, 128, s_pitch]")
+    iq, ik, iv = (float(x) for x in inv_scales)
+    _check(load_library().wan_quantize_fp8(_bf16_cuda(qkv, "qkv"), _u8_cuda(qk8, "qk8"), _u8_cuda(v8t, "v8t"), B, S,
+                                           heads, HEAD_DIM, v8t.shape[3], iq, ik, iv, _stream(stream)),
+           "wan_quantize_fp8")
+    return qk8, v8t
+
+
+def self_attention_fp8(qk8, v8t, heads: int, scales, out=None, scale: float = 0.0, stream=None):
+    """FP8 attention on e4m3 codes (quantize_fp8) dequantised with `scales`
+    (scale_q, scale_k, scale_v): out bf16 [B, S, heads*128]."""
+    import torch
+    B, S, d2 = qk8.shape
+    if d2 != 2 * heads * HEAD_DIM or v8t.dim() != 4 or tuple(v8t.shape[:3]) != (B, heads, HEAD_DIM):
+        raise ValueError("qk8 must be [B, S, 2*heads*128] and v8t [B, heads, 128, s_pitch]")
+    if out is None:
+        out = torch.empty((B, S, heads * HEAD_DIM), dtype=torch.bfloat16, device=qk8.device)
+    if tuple(out.shape) != (B, S, heads * HEAD_DIM):
+        raise ValueError("out must be [B, S, heads*128]")
+    sq, sk, sv = (float(x) for x in scales)
+    _check(load_library().wan_self_attention_fp8(_u8_cuda(qk8, "qk8"), _u8_cuda(v8t, "v8t"), _bf16_cuda(out, "out"),
+                                                 B, S, heads, HEAD_DIM, v8t.shape[3], scale, sq, sk, sv,
+                                                 _stream(stream)), "wan_self_attention_fp8")
+    return out
 
 
 def dit_attn(qkv, grid: Sequence[int], heads: int, gamma_q, gamma_k, out=None, eps: float = EPS,

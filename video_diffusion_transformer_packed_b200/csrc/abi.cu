@@ -11,7 +11,7 @@
 
 namespace {
 
-constexpr int32_t kAbiVersion = 4;
+constexpr int32_t kAbiVersion = 5;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -186,6 +186,82 @@ int32_t wan_self_attention_sparse(const void* qkv, void* out, int64_t batch, int
   return WAN_OK;
 }
 
+int32_t wan_qkv_amax(const void* qkv, int64_t batch, int64_t seq_len, int32_t heads, int32_t head_dim,
+                     float* amax, void* stream) {
+  WAN_TRY(check_heads(heads, head_dim));
+  WAN_TRY(check_tokens(batch, seq_len, heads));
+  if (!qkv || !amax) return WAN_ERR_NULL;
+  if (!aligned16(qkv) || (reinterpret_cast<uintptr_t>(amax) & 3u)) return WAN_ERR_ALIGN;
+  WAN_TRY(check_device());
+  (void)cudaGetLastError();
+  if (wan::launch_qkv_amax(qkv, batch * seq_len, heads, amax, static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess) {
+    return WAN_ERR_LAUNCH;
+  }
+  return WAN_OK;
+}
+
+namespace {
+bool positive_finite(float x) { return std::isfinite(x) && x > 0.f; }
+bool overlaps(const void* a, uint64_t na, const void* b, uint64_t nb) {
+  const uint64_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + nb && b0 < a0 + na;
+}
+int32_t check_fp8_buffers(int64_t batch, int64_t S, int32_t heads, int64_t s_pitch, const void* qk8,
+                          const void* v8t, const void* other, uint64_t other_bytes) {
+  if (!qk8 || !v8t || !other) return WAN_ERR_NULL;
+  if (!aligned16(qk8) || !aligned16(v8t) || !aligned16(other)) return WAN_ERR_ALIGN;
+  if (s_pitch < S || s_pitch % 16 != 0 || s_pitch > (int64_t)INT32_MAX) return WAN_ERR_SHAPE;
+  const uint64_t d = static_cast<uint64_t>(heads) * WAN_HEAD_DIM;
+  const uint64_t qk_bytes = static_cast<uint64_t>(batch) * S * 2 * d;
+  const uint64_t vt_bytes = static_cast<uint64_t>(batch) * d * s_pitch;
+  if (overlaps(qk8, qk_bytes, v8t, vt_bytes) || overlaps(qk8, qk_bytes, other, other_bytes) ||
+      overlaps(v8t, vt_bytes, other, other_bytes)) {
+    return WAN_ERR_ALIAS;
+  }
+  return WAN_OK;
+}
+}  // namespace
+
+int32_t wan_quantize_fp8(const void* qkv, void* qk8, void* v8t, int64_t batch, int64_t seq_len, int32_t heads,
+                         int32_t head_dim, int64_t s_pitch, float inv_scale_q, float inv_scale_k,
+                         float inv_scale_v, void* stream) {
+  WAN_TRY(check_heads(heads, head_dim));
+  WAN_TRY(check_tokens(batch, seq_len, heads));
+  const uint64_t qkv_bytes = static_cast<uint64_t>(batch) * seq_len * 3 * heads * WAN_HEAD_DIM * 2;
+  WAN_TRY(check_fp8_buffers(batch, seq_len, heads, s_pitch, qk8, v8t, qkv, qkv_bytes));
+  if (!positive_finite(inv_scale_q) || !positive_finite(inv_scale_k) || !positive_finite(inv_scale_v)) {
+    return WAN_ERR_PARAM;
+  }
+  WAN_TRY(check_device());
+  (void)cudaGetLastError();
+  if (wan::launch_quantize_fp8(qkv, qk8, v8t, batch, seq_len, heads, s_pitch, inv_scale_q, inv_scale_k,
+                               inv_scale_v, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    return WAN_ERR_LAUNCH;
+  }
+  return WAN_OK;
+}
+
+int32_t wan_self_attention_fp8(const void* qk8, const void* v8t, void* out, int64_t batch, int64_t seq_len,
+                               int32_t heads, int32_t head_dim, int64_t s_pitch, float scale, float scale_q,
+                               float scale_k, float scale_v, void* stream) {
+  WAN_TRY(check_heads(heads, head_dim));
+  WAN_TRY(check_tokens(batch, seq_len, heads));
+  const uint64_t out_bytes = static_cast<uint64_t>(batch) * seq_len * heads * WAN_HEAD_DIM * 2;
+  WAN_TRY(check_fp8_buffers(batch, seq_len, heads, s_pitch, qk8, v8t, out, out_bytes));
+  if (!std::isfinite(scale) || !positive_finite(scale_q) || !positive_finite(scale_k) ||
+      !positive_finite(scale_v)) {
+    return WAN_ERR_PARAM;
+  }
+  WAN_TRY(check_device());
+  (void)cudaGetLastError();
+  if (wan::launch_attn_fp8(qk8, v8t, out, batch, seq_len, heads, s_pitch, scale, scale_q, scale_k, scale_v,
+                           static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    return WAN_ERR_LAUNCH;
+  }
+  return WAN_OK;
+}
+
 int32_t wan_skip_stats(void* stream, int64_t* group_tiles, int64_t* products) {
   int64_t g = 0, pr = 0;
   if (wan::read_and_clear_skip_stats(static_cast<cudaStream_t>(stream), &g, &pr) != cudaSuccess) {
@@ -283,12 +359,13 @@ int32_t wan_selftest_wait_timeout(const void* qkv, void* out, int64_t batch, int
 int32_t wan_device_error(void* stream, int32_t* code) {
   if (!code) return WAN_ERR_NULL;
   *code = 0;
-  int32_t attn = 0, norm = 0;
+  int32_t attn = 0, norm = 0, fp8 = 0;
   if (wan::read_and_clear_device_error(static_cast<cudaStream_t>(stream), &attn) != cudaSuccess ||
-      wan::read_and_clear_norm_error(static_cast<cudaStream_t>(stream), &norm) != cudaSuccess) {
+      wan::read_and_clear_norm_error(static_cast<cudaStream_t>(stream), &norm) != cudaSuccess ||
+      wan::read_and_clear_fp8_error(static_cast<cudaStream_t>(stream), &fp8) != cudaSuccess) {
     return WAN_ERR_LAUNCH;
   }
-  *code = attn | (norm << 8);
+  *code = attn | (norm << 8) | (fp8 << 16);
   return *code != 0 ? WAN_ERR_DEVICE_TIMEOUT : WAN_OK;
 }
 

@@ -57,6 +57,19 @@ struct HostStep {
 };
 cudaError_t enqueue_dit_attn_host(const HostStep& step, cudaStream_t stream);
 
+// FP8 (e4m3) variant (fp8_quant.cu, attn_fwd_fp8.cu). Codes of X are
+// e4m3(fl32(x * inv_X)); the attention dequantises with scale_X. qk8 is
+// [B][S][2D] (Q then K codes of each token), v8t [B][heads][128][s_pitch]
+// (V codes transposed, zero past S; s_pitch a multiple of 16, >= S).
+cudaError_t launch_quantize_fp8(const void* qkv, void* qk8, void* v8t, int64_t batch, int64_t S,
+                                int32_t heads, int64_t s_pitch, float inv_q, float inv_k, float inv_v,
+                                cudaStream_t stream);
+cudaError_t launch_qkv_amax(const void* qkv, int64_t tokens, int32_t heads, float* amax, cudaStream_t stream);
+cudaError_t launch_attn_fp8(const void* qk8, const void* v8t, void* out, int64_t batch, int64_t seq_len,
+                            int32_t heads, int64_t s_pitch, float scale, float scale_q, float scale_k,
+                            float scale_v, cudaStream_t stream);
+cudaError_t read_and_clear_fp8_error(cudaStream_t stream, int32_t* code);
+
 // Synchronise the stream, then read and clear the Skip-Softmax counters:
 // (32-row group, key tile) pairs skipped, and P V products skipped.
 cudaError_t read_and_clear_skip_stats(cudaStream_t stream, int64_t* group_tiles, int64_t* products);

@@ -57,6 +57,7 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-skip", action="store_true", help="skip the Skip-Softmax side measurement")
+    ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 side measurement")
     return ap.parse_args()
 
 
@@ -386,6 +387,45 @@ def run_ours(args):
                                    "products_skipped": prods / (w.batch * w.heads * n_t * n_t)})
         del loc
 
+    # ---- FP8 (e4m3) side measurement (not the headline): the normalised
+    # buffer of a step, per-tensor scales amax/448, the quantisation and the
+    # FP8 attention timed separately, and the FP8 output's divergence from
+    # the bf16 kernel's on the same buffer.
+    fp8 = None
+    if not args.no_fp8:
+        src = bufs[0]  # normalised by the per-kernel pass above
+        amax_d = wan.qkv_amax(src, w.heads, stream=stream)
+        stream.synchronize()  # the maxima are written on `stream`; read them only after it
+        amax = amax_d.cpu().numpy().astype("float32")
+        sc = [float(a) / 448.0 for a in amax]
+        inv = [448.0 / float(a) for a in amax]
+        qk8, v8t = wan.quantize_fp8(src, w.heads, inv, stream=stream)
+        out8 = torch.empty_like(out)
+        wan.self_attention_fp8(qk8, v8t, w.heads, sc, out=out8, stream=stream)
+        wan.self_attention(src, w.heads, out=out, stream=stream)
+        stream.synchronize()
+        rel = float((out8.float() - out.float()).norm() / out.float().norm())
+
+        def timed_ms(fn, reps=3):
+            fn()
+            a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(reps):
+                fn()
+            b_.record(stream)
+            b_.synchronize()
+            return a.elapsed_time(b_) / reps
+
+        q_ms = timed_ms(lambda: wan.quantize_fp8(src, w.heads, inv, qk8, v8t, stream=stream))
+        a_ms = timed_ms(lambda: wan.self_attention_fp8(qk8, v8t, w.heads, sc, out=out8, stream=stream))
+        if wan.device_error(stream) != 0:
+            raise SystemExit("FP8 attention reported a device timeout")
+        fp8 = {"scales": "per tensor, amax/448", "quantize_ms": q_ms, "attention_ms": a_ms,
+               "attn_tflops_equiv": w.attn_flop / (a_ms / 1e3) / 1e12,
+               "path_tflops_equiv": w.attn_flop / ((q_ms + a_ms) / 1e3) / 1e12,
+               "rel_fro_vs_bf16": rel}
+        del qk8, v8t, out8
+
     peaks, peak_src = load_peaks()
     tensor_peak = peaks["bf16_tflops_sustained"]
     roofline = {
@@ -427,7 +467,7 @@ def run_ours(args):
         "attn_tflops": attn_tflops, "attn_frac_of_peak": attn_tflops / tensor_peak,
         "norm_rope_gbs": norm_gbs, "norm_rope_frac_of_hbm": norm_gbs / peaks["hbm_gbs"],
         "roofline": roofline, "roofline_norm_rope": norm_roofline,
-        "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks, "skip_softmax": skip,
+        "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks, "skip_softmax": skip, "fp8": fp8,
         "gpu_launches": 2 * args.steps,
     }
     print(json.dumps(line), flush=True)

@@ -191,7 +191,8 @@ def _u8_cuda(t, name: str) -> int:
 
 
 def qkv_amax(qkv, heads: int, stream=None):
-    """max |x| of Q, K and V of a packed bf16 buffer: float32 CUDA tensor [3]."""
+    """max |x| of Q, K and V of a packed bf16 buffer: float32 CUDA tensor [3],
+    written asynchronously on `stream` (synchronise it before reading)."""
     import torch
     _check_packed(qkv, heads)
     B, S, _ = qkv.shape

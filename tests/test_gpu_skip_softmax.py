@@ -119,3 +119,36 @@ def test_skipping_really_skips_products():
     groups, _, sk, margin = oracle_groups(qkv_h, heads, 0.05)
     assert (margin > MARGIN).all()
     assert (tiles, products) == expected_counts(groups, sk, S)
+
+
+def test_skip_softmax_full_size_sampled_groups():
+    """The bench shape (2 x 32760 tokens, 40 heads) with local peaked inputs at
+    threshold 0.05, in the bench's launch configuration: sampled 32-row groups
+    (the first, the last -- ragged, so never skipping -- and random ones)
+    against the oracle's skip-aware reference, where its decisions are clear."""
+    import wan_inputs as wi_
+    w = wi_.BY_NAME["a14b_480p_81f_cfg_b2"]
+    qkv = local_qkv(w.batch, w.seq_len, w.heads, seed=5)
+    wan.skip_stats()
+    out = wan.self_attention_sparse(qkv.cuda(), w.heads, 0.05)
+    tiles, products = wan.skip_stats()
+    assert products > 0
+    n_groups = (w.seq_len + 31) // 32
+    g = torch.Generator().manual_seed(11)
+    groups = [(0, 0, 0), (w.batch - 1, w.heads - 1, n_groups - 1)] + [
+        (int(torch.randint(w.batch, (1,), generator=g)), int(torch.randint(w.heads, (1,), generator=g)),
+         int(torch.randint(n_groups, (1,), generator=g))) for _ in range(4)]
+    ref, sk, margin = oracle.attention_skip_groups(qkv, w.heads, groups, SCALE, 0.05)
+    assert not sk[1].any()  # the ragged last group never skips
+    assert sk[2:].any()      # random groups do skip
+    oc = out.cpu().float().view(w.batch, w.seq_len, w.heads, HD)
+    gots, refs = [], []
+    for (b, h, gg), o, m in zip(groups, ref, margin):
+        if m <= MARGIN:
+            continue
+        n = min(32, w.seq_len - 32 * gg)
+        gots.append(oc[b, 32 * gg:32 * gg + n, h].numpy())
+        refs.append(o[:n])
+    assert len(gots) >= 4
+    assert_attention_close(torch.from_numpy(np.concatenate(gots)), np.concatenate(refs), "skip full size",
+                           scaled=True)

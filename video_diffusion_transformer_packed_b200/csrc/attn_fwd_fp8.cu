@@ -247,6 +247,36 @@ __device__ void run_mma(const AttnFp8Params& p, uint32_t smem, Bars bars, volati
   if (!mbar_wait(bars.drain(), 0, nullptr, kWaitLimitNs)) atomicOr(&g_attn_fp8_error_word, kErrDrain);
 }
 
+// 2^x on the FMA pipe for a quarter of the exponentials (MUFU ex2 gives 16
+// per clock per SM, as many cycles per tile as the fp8 products need twice
+// over): x = n + f, n = round(x) by the 1.5*2^23 magic add, f in [-1/2, 1/2];
+// 2^x = 2^n * p(f) with p the degree-3 minimax fit of 2^f in relative error
+// (7.5e-5) that exp2_poly.py next to this file computes; 2^n is applied by
+// adding n to the exponent field. x is clamped at -126 (masked keys).
+constexpr uint32_t kPolyC0 = 0x3F7FFB49u, kPolyC1 = 0x3F31798Du, kPolyC2 = 0x3E786F0Du,
+                   kPolyC3 = 0x3D61FBB0u;
+constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
+  float x0, x1;
+  f2_split(x2, x0, x1);
+  x2 = f2(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+  const uint64_t magic = f2(kMagic, kMagic);
+  const uint64_t j = add2(x2, magic);
+  const uint64_t f = sub2(x2, sub2(j, magic));
+  uint64_t p = fma2(f2(__uint_as_float(kPolyC3), __uint_as_float(kPolyC3)), f,
+                    f2(__uint_as_float(kPolyC2), __uint_as_float(kPolyC2)));
+  p = fma2(p, f, f2(__uint_as_float(kPolyC1), __uint_as_float(kPolyC1)));
+  p = fma2(p, f, f2(__uint_as_float(kPolyC0), __uint_as_float(kPolyC0)));
+  float p0, p1, j0, j1;
+  f2_split(p, p0, p1);
+  f2_split(j, j0, j1);
+  const float r0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(j0) << 23));
+  const float r1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(j1) << 23));
+  return f2(r0, r1);
+}
+// Four-key groups whose exponentials take the polynomial: one in four.
+__host__ __device__ constexpr bool poly_group(int w) { return (w & 3) == 3; }
+
 // ----------------------------------------------------------------- softmax
 __device__ void run_softmax(const AttnFp8Params& p, Bars bars, volatile int* abort, uint32_t tmem, int t,
                             int quarter, int lane, int b, int h, int qp) {
@@ -316,10 +346,16 @@ __device__ void run_softmax(const AttnFp8Params& p, Bars bars, volatile int* abo
         const int k4 = 64 * part + 4 * w;
         const uint64_t xa = fma2(f2(__uint_as_float(sr[k4]), __uint_as_float(sr[k4 + 1])), sl2_2, negm2);
         const uint64_t xb = fma2(f2(__uint_as_float(sr[k4 + 2]), __uint_as_float(sr[k4 + 3])), sl2_2, negm2);
-        float x0, x1, x2, x3;
-        f2_split(xa, x0, x1);
-        f2_split(xb, x2, x3);
-        const float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(x2), p3 = ex2(x3);
+        float p0, p1, p2, p3;
+        if (poly_group(w)) {
+          f2_split(exp2_poly2(xa), p0, p1);
+          f2_split(exp2_poly2(xb), p2, p3);
+        } else {
+          float x0, x1, x2, x3;
+          f2_split(xa, x0, x1);
+          f2_split(xb, x2, x3);
+          p0 = ex2(x0); p1 = ex2(x1); p2 = ex2(x2); p3 = ex2(x3);
+        }
         sum2[(2 * w) & 3] = add2(sum2[(2 * w) & 3], f2(p0, p1));
         sum2[(2 * w + 1) & 3] = add2(sum2[(2 * w + 1) & 3], f2(p2, p3));
         pk[w] = pack_e4m3x4(p0, p1, p2, p3);

@@ -178,6 +178,31 @@ WAN_API int32_t wan_self_attention_fp8(const void* qk8, const void* v8t, void* o
                                        float scale, float scale_q, float scale_k, float scale_v, void* stream);
 
 /*
+ * The DiT block's projections (the third NEXT item): Y = X W^T on the tensor
+ * cores (tcgen05, bf16 operands, fp32 accumulation, bf16 output), X [M][K],
+ * W [N][K] (a Linear layer's weight), Y [M][N], all device, 16-byte aligned,
+ * N a multiple of 256, K a multiple of 64, Y overlapping neither input. For
+ * the QKV projection (N = 3*heads*128, Y the packed buffer) the epilogue can
+ * fuse the Q/K RMSNorm's statistic (the Neuron page's qkv_cte fuses the
+ * projection with the distributed QK RMSNorm, "NKI kernels"): when stats is
+ * not NULL, stats[row][j] = the fp64 sum of squares of the bf16 outputs of
+ * row `row` in columns [256 j, 256 j + 256), for j < stat_cols / 256
+ * (stat_cols a multiple of 256, <= N; stats 8-byte aligned, [M][stat_cols/256]).
+ */
+WAN_API int32_t wan_linear(const void* x, const void* w, void* y, int64_t M, int64_t N, int64_t K,
+                           double* stats, int64_t stat_cols, void* stream);
+
+/*
+ * (1) with the row statistics of the QKV projection: as wan_qk_norm_rope, but
+ * each token's sum of squares of Q (and of K) is the sum of its stats entries
+ * (wan_linear with stat_cols = 2*heads*128 on the same buffer) instead of a
+ * reduction over the row. stats: device, [batch*F*H*W][2*heads*128/256] fp64.
+ */
+WAN_API int32_t wan_qk_norm_rope_stats(void* qkv, int64_t batch, int32_t F, int32_t H, int32_t W, int32_t heads,
+                                       int32_t head_dim, const void* gamma_q, const void* gamma_k, float eps,
+                                       float theta, const double* stats, void* stream);
+
+/*
  * Synchronises `stream`, then reads and clears the Skip-Softmax counters
  * accumulated by wan_self_attention_sparse launches since the last read:
  * *group_tiles = (32-row group, key tile) pairs skipped, *products = 128-row
@@ -240,7 +265,7 @@ WAN_API int32_t wan_dit_attn_host(const void* qkv_host, void* out_host, void* qk
  * that the kernels set when one of their bounded waits gives up. *code
  * receives 0 when no wait gave up, otherwise a nonzero value: the bf16
  * attention's site code in bits 0-7, norm+RoPE's in bits 8-15, the FP8
- * attention's in bits 16-23.
+ * attention's in bits 16-23, the projection GEMM's in bits 24-30.
  * Returns WAN_ERR_DEVICE_TIMEOUT when *code != 0, WAN_ERR_NULL when code is
  * NULL, WAN_ERR_LAUNCH when the synchronisation reports a CUDA error.
  */

@@ -215,6 +215,15 @@ def attention_fp8_rows(qk8: np.ndarray, v8t: np.ndarray, heads: int, rows, scale
     return out
 
 
+def linear_rows(x: torch.Tensor, w: torch.Tensor, rows) -> np.ndarray:
+    """The QKV (or output) projection Y = X W^T for listed rows of X [M, K]
+    (bf16 values, exact in fp64), in fp64 with numpy's matrix product: [n, N].
+    The projection precedes the path (TensorRT-LLM PR "[visual_gen] Optimize
+    Wan2.2 Dataflow": the fused QKV projection output is the packed buffer)."""
+    xr = x.reshape(-1, x.shape[-1])[torch.as_tensor(np.asarray(rows, dtype=np.int64))].double().numpy()
+    return xr @ w.double().numpy().T
+
+
 def attention_full(qkv: torch.Tensor, heads: int, scale: float) -> np.ndarray:
     """Step 4 for every row: fp64 [B, S, heads, 128]."""
     B, S, _ = qkv.shape

@@ -39,7 +39,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings(lib):
-    assert lib.wan_abi_version() == 5
+    assert lib.wan_abi_version() == 6
     for code in range(11):
         assert lib.wan_status_string(code)
     assert lib.wan_status_string(99) == b"unknown status"
@@ -159,3 +159,20 @@ def test_fp8_entry_points_validate(lib):
     import torch
     if not torch.cuda.is_available():
         assert lib.wan_self_attention_fp8(far1, far2, FAKE, 1, 8, 1, 128, 16, 0.0, 1.0, 1.0, 1.0, None) == 6
+
+
+def test_linear_validates(lib):
+    far = 2**40
+    # (x, w, y, M, N, K, stats, stat_cols)
+    assert lib.wan_linear(None, FAKE, far, 4, 256, 64, None, 0, None) == 1
+    assert lib.wan_linear(FAKE + 4, FAKE, far, 4, 256, 64, None, 0, None) == 2
+    assert lib.wan_linear(FAKE, FAKE, far, 4, 200, 64, None, 0, None) == 3   # N % 256
+    assert lib.wan_linear(FAKE, FAKE, far, 4, 256, 100, None, 0, None) == 3  # K % 64
+    assert lib.wan_linear(FAKE, FAKE, far, 4, 256, 64, 2**41, 512, None) == 3  # stat_cols > N
+    assert lib.wan_linear(FAKE, FAKE, far, 4, 256, 64, 2**41 + 4, 256, None) == 2
+    assert lib.wan_linear(FAKE, FAKE, FAKE + 64, 4, 256, 64, None, 0, None) == 9  # y overlaps x
+    assert lib.wan_qk_norm_rope_stats(FAKE, 1, 2, 2, 2, 2, 128, FAKE, FAKE, 1e-6, 1e4, None, None) == 1
+    assert lib.wan_qk_norm_rope_stats(FAKE, 1, 2, 2, 2, 1, 128, FAKE, FAKE, 1e-6, 1e4, 2**41, None) == 3  # D=128
+    import torch
+    if not torch.cuda.is_available():
+        assert lib.wan_linear(FAKE, FAKE, far, 4, 256, 64, None, 0, None) == 6

@@ -20,7 +20,7 @@ from typing import Optional, Sequence
 
 __all__ = ["WanError", "load_library", "library_path", "qk_norm_rope", "self_attention",
            "self_attention_sparse", "skip_stats", "qkv_amax", "quantize_fp8", "self_attention_fp8",
-           "fp8_pitch", "dit_attn", "dit_attn_host", "device_error", "selftest_wait_timeout", "HEAD_DIM", "EPS",
+           "fp8_pitch", "linear", "qk_norm_rope_stats", "dit_attn", "dit_attn_host", "device_error", "selftest_wait_timeout", "HEAD_DIM", "EPS",
            "THETA", "STATUS"]
 
 HEAD_DIM = 128
@@ -87,6 +87,10 @@ def load_library() -> ctypes.CDLL:
             lib.wan_quantize_fp8.restype = I32
             lib.wan_self_attention_fp8.argtypes = [P, P, P, I64, I64, I32, I32, I64, F, F, F, F, P]
             lib.wan_self_attention_fp8.restype = I32
+            lib.wan_linear.argtypes = [P, P, P, I64, I64, I64, P, I64, P]
+            lib.wan_linear.restype = I32
+            lib.wan_qk_norm_rope_stats.argtypes = [P, I64, I32, I32, I32, I32, I32, P, P, F, F, P, P]
+            lib.wan_qk_norm_rope_stats.restype = I32
             _lib = lib
     return _lib
 
@@ -242,6 +246,49 @@ def self_attention_fp8(qk8, v8t, heads: int, scales, out=None, scale: float = 0.
                                                  B, S, heads, HEAD_DIM, v8t.shape[3], scale, sq, sk, sv,
                                                  _stream(stream)), "wan_self_attention_fp8")
     return out
+
+
+def linear(x, w, y=None, stat_cols: int = 0, stream=None):
+    """Y = X W^T (bf16, fp32 accumulation) for X [..., K] and W [N, K]; with
+    stat_cols > 0 also returns the fp64 sums of squares of the bf16 outputs per
+    row and 256-column tile of the first stat_cols columns: (y, stats) with
+    stats [M, stat_cols // 256], else (y, None)."""
+    import torch
+    K = x.shape[-1]
+    M = x.numel() // K
+    N = w.shape[0]
+    if w.dim() != 2 or w.shape[1] != K:
+        raise ValueError(f"w must be [N, {K}], got {tuple(w.shape)}")
+    if y is None:
+        y = torch.empty((*x.shape[:-1], N), dtype=torch.bfloat16, device=x.device)
+    if y.numel() != M * N:
+        raise ValueError("y must hold M x N elements")
+    stats = None
+    if stat_cols:
+        stats = torch.empty((M, stat_cols // 256), dtype=torch.float64, device=x.device)
+    _check(load_library().wan_linear(_bf16_cuda(x, "x"), _bf16_cuda(w, "w"), _bf16_cuda(y, "y"), M, N, K,
+                                     stats.data_ptr() if stats is not None else None, int(stat_cols),
+                                     _stream(stream)), "wan_linear")
+    return y, stats
+
+
+def qk_norm_rope_stats(qkv, grid: Sequence[int], heads: int, gamma_q, gamma_k, stats, eps: float = EPS,
+                       theta: float = THETA, stream=None):
+    """qk_norm_rope taking each token's sums of squares from the QKV
+    projection's statistics (linear(..., stat_cols=2*heads*128))."""
+    import torch
+    F, H, W = grid
+    B = qkv.shape[0]
+    _check_packed(qkv, heads, grid)
+    _check_gamma(gamma_q, heads, "gamma_q")
+    _check_gamma(gamma_k, heads, "gamma_k")
+    if stats.dtype != torch.float64 or not stats.is_cuda or tuple(stats.shape) != (B * qkv.shape[1], 2 * heads * HEAD_DIM // 256):
+        raise ValueError("stats must be float64 CUDA [B*S, 2*heads*128/256]")
+    _check(load_library().wan_qk_norm_rope_stats(_bf16_cuda(qkv, "qkv"), B, F, H, W, heads, HEAD_DIM,
+                                                 _bf16_cuda(gamma_q, "gamma_q"), _bf16_cuda(gamma_k, "gamma_k"),
+                                                 eps, theta, stats.data_ptr(), _stream(stream)),
+           "wan_qk_norm_rope_stats")
+    return qkv
 
 
 def dit_attn(qkv, grid: Sequence[int], heads: int, gamma_q, gamma_k, out=None, eps: float = EPS,

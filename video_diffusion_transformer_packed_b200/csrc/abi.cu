@@ -11,7 +11,7 @@
 
 namespace {
 
-constexpr int32_t kAbiVersion = 5;
+constexpr int32_t kAbiVersion = 6;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -101,6 +101,12 @@ int32_t check_memory_kind(const void* host_in, const void* host_out, const void*
     if (at.type != cudaMemoryTypeDevice || at.device != dev) return WAN_ERR_MEMORY_KIND;
   }
   return WAN_OK;
+}
+
+bool positive_finite(float x) { return std::isfinite(x) && x > 0.f; }
+bool overlaps(const void* a, uint64_t na, const void* b, uint64_t nb) {
+  const uint64_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + nb && b0 < a0 + na;
 }
 
 #define WAN_TRY(expr)          \
@@ -202,11 +208,6 @@ int32_t wan_qkv_amax(const void* qkv, int64_t batch, int64_t seq_len, int32_t he
 }
 
 namespace {
-bool positive_finite(float x) { return std::isfinite(x) && x > 0.f; }
-bool overlaps(const void* a, uint64_t na, const void* b, uint64_t nb) {
-  const uint64_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
-  return a0 < b0 + nb && b0 < a0 + na;
-}
 int32_t check_fp8_buffers(int64_t batch, int64_t S, int32_t heads, int64_t s_pitch, const void* qk8,
                           const void* v8t, const void* other, uint64_t other_bytes) {
   if (!qk8 || !v8t || !other) return WAN_ERR_NULL;
@@ -257,6 +258,46 @@ int32_t wan_self_attention_fp8(const void* qk8, const void* v8t, void* out, int6
   (void)cudaGetLastError();
   if (wan::launch_attn_fp8(qk8, v8t, out, batch, seq_len, heads, s_pitch, scale, scale_q, scale_k, scale_v,
                            static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    return WAN_ERR_LAUNCH;
+  }
+  return WAN_OK;
+}
+
+int32_t wan_linear(const void* x, const void* w, void* y, int64_t M, int64_t N, int64_t K, double* stats,
+                   int64_t stat_cols, void* stream) {
+  if (!x || !w || !y) return WAN_ERR_NULL;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(y)) return WAN_ERR_ALIGN;
+  if (stats && (reinterpret_cast<uintptr_t>(stats) & 7u)) return WAN_ERR_ALIGN;
+  if (M < 1 || N < 256 || K < 64 || N % 256 != 0 || K % 64 != 0) return WAN_ERR_SHAPE;
+  if (M > (1LL << 31) || N > (1LL << 24) || K > (1LL << 24)) return WAN_ERR_SHAPE;
+  if (stats && (stat_cols < 256 || stat_cols % 256 != 0 || stat_cols > N)) return WAN_ERR_SHAPE;
+  const uint64_t xb = static_cast<uint64_t>(M) * K * 2, wb = static_cast<uint64_t>(N) * K * 2;
+  const uint64_t yb = static_cast<uint64_t>(M) * N * 2;
+  if (overlaps(y, yb, x, xb) || overlaps(y, yb, w, wb)) return WAN_ERR_ALIAS;
+  if (stats && overlaps(stats, static_cast<uint64_t>(M) * (stat_cols / 256) * 8, y, yb)) return WAN_ERR_ALIAS;
+  WAN_TRY(check_device());
+  (void)cudaGetLastError();
+  if (wan::launch_gemm_bf16(x, w, y, M, N, K, stats, stats ? stat_cols : 0, static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess) {
+    return WAN_ERR_LAUNCH;
+  }
+  return WAN_OK;
+}
+
+int32_t wan_qk_norm_rope_stats(void* qkv, int64_t batch, int32_t F, int32_t H, int32_t W, int32_t heads,
+                               int32_t head_dim, const void* gamma_q, const void* gamma_k, float eps, float theta,
+                               const double* stats, void* stream) {
+  int64_t S = 0;
+  WAN_TRY(check_heads(heads, head_dim));
+  WAN_TRY(check_grid(batch, F, H, W, heads, &S));
+  WAN_TRY(check_norm_args(qkv, gamma_q, gamma_k, eps, theta));
+  if (!stats) return WAN_ERR_NULL;
+  if (reinterpret_cast<uintptr_t>(stats) & 7u) return WAN_ERR_ALIGN;
+  if ((heads * WAN_HEAD_DIM) % 256 != 0) return WAN_ERR_SHAPE;  // whole 256-column statistic tiles
+  WAN_TRY(check_device());
+  (void)cudaGetLastError();
+  if (wan::launch_qk_norm_rope(qkv, batch, F, H, W, heads, gamma_q, gamma_k, eps, theta,
+                               static_cast<cudaStream_t>(stream), stats) != cudaSuccess) {
     return WAN_ERR_LAUNCH;
   }
   return WAN_OK;
@@ -359,13 +400,14 @@ int32_t wan_selftest_wait_timeout(const void* qkv, void* out, int64_t batch, int
 int32_t wan_device_error(void* stream, int32_t* code) {
   if (!code) return WAN_ERR_NULL;
   *code = 0;
-  int32_t attn = 0, norm = 0, fp8 = 0;
+  int32_t attn = 0, norm = 0, fp8 = 0, gemm = 0;
   if (wan::read_and_clear_device_error(static_cast<cudaStream_t>(stream), &attn) != cudaSuccess ||
       wan::read_and_clear_norm_error(static_cast<cudaStream_t>(stream), &norm) != cudaSuccess ||
-      wan::read_and_clear_fp8_error(static_cast<cudaStream_t>(stream), &fp8) != cudaSuccess) {
+      wan::read_and_clear_fp8_error(static_cast<cudaStream_t>(stream), &fp8) != cudaSuccess ||
+      wan::read_and_clear_gemm_error(static_cast<cudaStream_t>(stream), &gemm) != cudaSuccess) {
     return WAN_ERR_LAUNCH;
   }
-  *code = attn | (norm << 8) | (fp8 << 16);
+  *code = attn | (norm << 8) | (fp8 << 16) | ((gemm & 0x7F) << 24);
   return *code != 0 ? WAN_ERR_DEVICE_TIMEOUT : WAN_OK;
 }
 

@@ -76,6 +76,11 @@ struct NormRopeParams {
   uint32_t stage_bytes;  // Q row + K row = 4 * D bytes
   double eps;
   double inv_d;
+  // Optional sums of squares from the QKV projection's epilogue
+  // (gemm_bf16.cu): stats[token][j], j < stat_row; Q's partials are
+  // j < stat_half, K's the next stat_half. Used by the kStats instantiation.
+  const double* stats;
+  int32_t stat_row, stat_half;
   double freq_pi[kPairs];  // per pair of a head: theta^(-2j/d_axis) / pi
 };
 
@@ -225,7 +230,7 @@ __device__ __forceinline__ void rotate2(uint32_t& wa, uint32_t& wb, const float4
   wb = wan::sm100::pack_bf16x2(e1, o1);
 }
 
-template <int VPT>
+template <int VPT, bool kStats>
 __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const __grid_constant__ NormRopeParams p) {
   using namespace wan::sm100;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -274,6 +279,12 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const __grid_
   int64_t i = 0;
   for (int64_t tok = blockIdx.x; tok < p.tokens; tok += step, ++i) {
     const int buf = static_cast<int>(i & 1);
+    // With precomputed statistics, lane j of each warp fetches the row's j-th
+    // partial sum now; the load's latency hides behind the ring wait.
+    double st_part = 0.0;
+    if constexpr (kStats) {
+      if (lane < p.stat_half) st_part = p.stats[tok * p.stat_row + which * p.stat_half + lane];
+    }
     // The next token's rotations, ahead of time (they do not depend on the data).
     const int rnext = rbuf == 2 ? 0 : rbuf + 1;
     if ((tid & 3) == 0 && tok + step < p.tokens) rotation(p, s_next, my_pr, tail.rot[rnext]);
@@ -291,18 +302,20 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const __grid_
       v[k] = vi < p.nvec ? ld_shared_v4(src + 16 * vi) : make_uint4(0, 0, 0, 0);
     }
 
-    double acc[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
+    if constexpr (!kStats) {
+      double acc[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
 #pragma unroll
-    for (int k = 0; k < VPT; ++k) {
-      sumsq_pair(v[k].x, acc[0], acc[1]);
-      sumsq_pair(v[k].y, acc[2], acc[3]);
-      sumsq_pair(v[k].z, acc[4], acc[5]);
-      sumsq_pair(v[k].w, acc[6], acc[7]);
+      for (int k = 0; k < VPT; ++k) {
+        sumsq_pair(v[k].x, acc[0], acc[1]);
+        sumsq_pair(v[k].y, acc[2], acc[3]);
+        sumsq_pair(v[k].z, acc[4], acc[5]);
+        sumsq_pair(v[k].w, acc[6], acc[7]);
+      }
+      double ss = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      if (lane == 0) tail.partial[buf][warp] = ss;
     }
-    double ss = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    if (lane == 0) tail.partial[buf][warp] = ss;
     __syncthreads();  // the stage is consumed; partial sums and rotations are visible
     if (tail.abort) break;
 
@@ -317,8 +330,17 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const __grid_
       }
     }
 
-    const double* part = &tail.partial[buf][4 * which];
-    const double rd = rsqrt(((part[0] + part[1]) + (part[2] + part[3])) * p.inv_d + p.eps);
+    double total;
+    if constexpr (kStats) {
+      // the same fixed tree in every warp: every thread gets the same sum
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) st_part += __shfl_xor_sync(0xffffffffu, st_part, o);
+      total = st_part;
+    } else {
+      const double* part = &tail.partial[buf][4 * which];
+      total = (part[0] + part[1]) + (part[2] + part[3]);
+    }
+    const double rd = rsqrt(total * p.inv_d + p.eps);
     const float r_hi = static_cast<float>(rd);
     const float r_lo = static_cast<float>(rd - static_cast<double>(r_hi));
     const uint64_t r2 = f2(r_hi, r_hi);
@@ -387,16 +409,16 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const __grid_
   grid_launch_dependents();
 }
 
-template <int VPT>
+template <int VPT, bool kStats>
 cudaError_t launch_vpt(const NormRopeParams& p, uint32_t smem_bytes, cudaStream_t stream) {
   static int blocks_per_sm = -1;  // per instantiation; the smem size is fixed per instantiation
   static uint32_t configured_smem = 0;
   if (configured_smem != smem_bytes) {
-    cudaError_t e = cudaFuncSetAttribute(qk_norm_rope_kernel<VPT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(qk_norm_rope_kernel<VPT, kStats>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem_bytes));
     if (e != cudaSuccess) return e;
     int n = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, qk_norm_rope_kernel<VPT>, kThreads, smem_bytes);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, qk_norm_rope_kernel<VPT, kStats>, kThreads, smem_bytes);
     if (e != cudaSuccess) return e;
     blocks_per_sm = n > 0 ? n : 1;
     configured_smem = smem_bytes;
@@ -407,15 +429,29 @@ cudaError_t launch_vpt(const NormRopeParams& p, uint32_t smem_bytes, cudaStream_
   if (e != cudaSuccess) return e;
   const int64_t want = static_cast<int64_t>(sms) * blocks_per_sm;
   const int64_t blocks = p.tokens < want ? p.tokens : want;
-  qk_norm_rope_kernel<VPT><<<static_cast<unsigned>(blocks), kThreads, smem_bytes, stream>>>(p);
+  qk_norm_rope_kernel<VPT, kStats><<<static_cast<unsigned>(blocks), kThreads, smem_bytes, stream>>>(p);
   return cudaGetLastError();
 }
 
 }  // namespace
 
+template <bool kStats>
+cudaError_t launch_vpt_dispatch(int vpt, const NormRopeParams& p, uint32_t smem_bytes, cudaStream_t stream) {
+  switch (vpt) {
+    case 1: return launch_vpt<1, kStats>(p, smem_bytes, stream);
+    case 2: return launch_vpt<2, kStats>(p, smem_bytes, stream);
+    case 3: return launch_vpt<3, kStats>(p, smem_bytes, stream);
+    case 4: return launch_vpt<4, kStats>(p, smem_bytes, stream);
+    case 5: return launch_vpt<5, kStats>(p, smem_bytes, stream);
+    case 6: return launch_vpt<6, kStats>(p, smem_bytes, stream);
+    case 7: return launch_vpt<7, kStats>(p, smem_bytes, stream);
+    default: return launch_vpt<8, kStats>(p, smem_bytes, stream);
+  }
+}
+
 cudaError_t launch_qk_norm_rope(void* qkv, int64_t batch, int32_t F, int32_t H, int32_t W,
                                 int32_t heads, const void* gamma_q, const void* gamma_k, float eps,
-                                float theta, cudaStream_t stream) {
+                                float theta, cudaStream_t stream, const double* stats) {
   NormRopeParams p;
   p.qkv = static_cast<uint16_t*>(qkv);
   p.gamma_q = static_cast<const uint16_t*>(gamma_q);
@@ -431,6 +467,9 @@ cudaError_t launch_qk_norm_rope(void* qkv, int64_t batch, int32_t F, int32_t H, 
   p.stages = stages < 2 ? 2 : (stages > kMaxStages ? kMaxStages : stages);
   p.eps = static_cast<double>(eps);
   p.inv_d = 1.0 / static_cast<double>(p.D);
+  p.stats = stats;
+  p.stat_half = p.D / 256;
+  p.stat_row = 2 * p.stat_half;
   const int split[3] = {44, 42, 42};
   for (int pr = 0; pr < kPairs; ++pr) {
     const int axis = pr < kRowAxisPair0 ? 0 : (pr < kColAxisPair0 ? 1 : 2);
@@ -441,16 +480,8 @@ cudaError_t launch_qk_norm_rope(void* qkv, int64_t batch, int32_t F, int32_t H, 
   if (p.tokens == 0) return cudaSuccess;
   const uint32_t smem_bytes = p.stages * p.stage_bytes + static_cast<uint32_t>(sizeof(NormSmemTail));
   const int vpt = (p.nvec + kRowThreads - 1) / kRowThreads;  // 16-byte vectors per thread
-  switch (vpt) {
-    case 1: return launch_vpt<1>(p, smem_bytes, stream);
-    case 2: return launch_vpt<2>(p, smem_bytes, stream);
-    case 3: return launch_vpt<3>(p, smem_bytes, stream);
-    case 4: return launch_vpt<4>(p, smem_bytes, stream);
-    case 5: return launch_vpt<5>(p, smem_bytes, stream);
-    case 6: return launch_vpt<6>(p, smem_bytes, stream);
-    case 7: return launch_vpt<7>(p, smem_bytes, stream);
-    default: return launch_vpt<8>(p, smem_bytes, stream);
-  }
+  if (stats != nullptr) return launch_vpt_dispatch<true>(vpt, p, smem_bytes, stream);
+  return launch_vpt_dispatch<false>(vpt, p, smem_bytes, stream);
 }
 
 cudaError_t read_and_clear_norm_error(cudaStream_t stream, int32_t* code) {

@@ -9,9 +9,12 @@ namespace wan {
 
 // Q/K RMSNorm + bf16 round + 3D RoPE, in place on the packed buffer.
 // Arguments are assumed validated by the ABI layer.
+// With `stats` (the QKV projection's per-256-column sums of squares of the
+// same buffer, [batch*S][2*heads*128/256] fp64, see launch_gemm_bf16) the kernel
+// takes each row's sum from them instead of reducing it.
 cudaError_t launch_qk_norm_rope(void* qkv, int64_t batch, int32_t F, int32_t H, int32_t W,
                                 int32_t heads, const void* gamma_q, const void* gamma_k, float eps,
-                                float theta, cudaStream_t stream);
+                                float theta, cudaStream_t stream, const double* stats = nullptr);
 
 // Everything the attention launch needs, prepared before anything is
 // launched (tensor-map encoding can fail; a launch after a successful plan
@@ -69,6 +72,14 @@ cudaError_t launch_attn_fp8(const void* qk8, const void* v8t, void* out, int64_t
                             int32_t heads, int64_t s_pitch, float scale, float scale_q, float scale_k,
                             float scale_v, cudaStream_t stream);
 cudaError_t read_and_clear_fp8_error(cudaStream_t stream, int32_t* code);
+
+// Y[M][N] = X[M][K] W[N][K]^T in bf16 with fp32 accumulation (gemm_bf16.cu);
+// N a multiple of 256, K of 64. When stats is not null, stats[row][j] (row
+// length stat_cols / 256) receives the fp64 sum of squares of the bf16 outputs
+// of row `row` in columns [256 j, 256 j + 256), for j < stat_cols / 256.
+cudaError_t launch_gemm_bf16(const void* x, const void* w, void* y, int64_t M, int64_t N, int64_t K,
+                             double* stats, int64_t stat_cols, cudaStream_t stream);
+cudaError_t read_and_clear_gemm_error(cudaStream_t stream, int32_t* code);
 
 // Synchronise the stream, then read and clear the Skip-Softmax counters:
 // (32-row group, key tile) pairs skipped, and P V products skipped.

@@ -58,6 +58,7 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-skip", action="store_true", help="skip the Skip-Softmax side measurement")
     ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 side measurement")
+    ap.add_argument("--no-proj", action="store_true", help="skip the QKV projection side measurement")
     return ap.parse_args()
 
 
@@ -426,6 +427,50 @@ def run_ours(args):
                "rel_fro_vs_bf16": rel}
         del qk8, v8t, out8
 
+    # ---- QKV projection side measurement (not the headline): the GEMM that
+    # produces the packed buffer (tokens x D -> tokens x 3D, seeded synthetic
+    # activations and weights), with and without its norm statistic, cuBLAS
+    # on the same operands for reference, and norm+RoPE fed by the statistic
+    # against the reducing kernel on the same buffer.
+    proj = None
+    if not args.no_proj:
+        M, D = w.batch * w.seq_len, w.dim
+        gen = torch.Generator(device=dev).manual_seed(11)
+        xact = torch.randn(M, D, device=dev, generator=gen).to(torch.bfloat16)
+        wqkv = (torch.randn(3 * D, D, device=dev, generator=gen) / D ** 0.5).to(torch.bfloat16)
+        yqkv = bufs[0]
+
+        def timed_p(fn, reps=3):
+            fn()
+            a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(reps):
+                fn()
+            b_.record(stream)
+            b_.synchronize()
+            return a.elapsed_time(b_) / reps
+
+        g_ms = timed_p(lambda: wan.linear(xact, wqkv, yqkv, stream=stream))
+        stats_box = {}
+
+        def with_stats():
+            _, stats_box["s"] = wan.linear(xact, wqkv, yqkv, stat_cols=2 * D, stream=stream)
+
+        gs_ms = timed_p(with_stats)
+        with torch.cuda.stream(stream):
+            cb_ms = timed_p(lambda: torch.matmul(xact, wqkv.t(), out=yqkv.view(M, 3 * D)))
+        with_stats()
+        ns_ms = timed_p(lambda: wan.qk_norm_rope_stats(yqkv, w.grid, w.heads, gq, gk, stats_box["s"], stream=stream))
+        n_ms = timed_p(lambda: wan.qk_norm_rope(yqkv, w.grid, w.heads, gq, gk, stream=stream))
+        if wan.device_error(stream) != 0:
+            raise SystemExit("projection kernels reported a device timeout")
+        pflop = 2.0 * M * D * 3 * D
+        proj = {"shape": f"{M} x {D} -> {3 * D}", "gemm_ms": g_ms, "gemm_tflops": pflop / (g_ms / 1e3) / 1e12,
+                "gemm_with_stats_ms": gs_ms, "cublas_ms": cb_ms, "cublas_tflops": pflop / (cb_ms / 1e3) / 1e12,
+                "norm_from_stats_ms": ns_ms, "norm_from_stats_gbs": w.norm_rope_bytes / (ns_ms / 1e3) / 1e9,
+                "norm_reducing_ms": n_ms}
+        del xact, wqkv, stats_box
+
     peaks, peak_src = load_peaks()
     tensor_peak = peaks["bf16_tflops_sustained"]
     roofline = {
@@ -468,6 +513,7 @@ def run_ours(args):
         "norm_rope_gbs": norm_gbs, "norm_rope_frac_of_hbm": norm_gbs / peaks["hbm_gbs"],
         "roofline": roofline, "roofline_norm_rope": norm_roofline,
         "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks, "skip_softmax": skip, "fp8": fp8,
+        "qkv_projection": proj,
         "gpu_launches": 2 * args.steps,
     }
     print(json.dumps(line), flush=True)

@@ -185,9 +185,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
+        bool ready = false;  // probe result for the stage of step `it`
         for (int ks = 0; ks < p.k_steps; ++ks, ++it) {
           const int slot = static_cast<int>(it % kStages);
-          if (!mbar_wait(bars.full(slot), static_cast<uint32_t>((it / kStages) & 1), abort, kWaitLimitNs)) {
+          if (!ready && !mbar_wait(bars.full(slot), static_cast<uint32_t>((it / kStages) & 1), abort, kWaitLimitNs)) {
             ok = false;
             break;
           }
@@ -198,6 +199,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < kKStep / 16; ++kk) {
             const uint32_t acc = (ks > 0 || kk > 0) ? 1u : 0u;
+            if (kk == kKStep / 16 - 1) {
+              // probe the next step's stage while this step's last MMAs wait for queue room
+              const int64_t nx = it + 1;
+              ready = ks + 1 < p.k_steps &&
+                      mbar_test(bars.full(static_cast<int>(nx % kStages)), static_cast<uint32_t>((nx / kStages) & 1));
+            }
             mma_ss(tmem, desc_add(desc0, a0 + 2 * kk), desc_add(desc0, b0 + 2 * kk), kIdesc, acc);
             mma_ss(tmem + 256, desc_add(desc0, a1 + 2 * kk), desc_add(desc0, b0 + 2 * kk), kIdesc, acc);
           }
@@ -240,12 +247,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             w[e] = pack_bf16x2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
           }
           if (stat) {
-            // squares of bf16 values are exact in fp32; their sum in fp64
+            // squares of bf16 values are exact in fp32 (16-bit significands)
+            // and move to fp64 by bit arithmetic: high word (bits >> 3) +
+            // ((1023 - 127) << 20), low word 0. A zero square maps to 2^-127
+            // (as in the norm kernel's own sum), negligible next to eps.
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
               const float lo = __uint_as_float(w[e] << 16), hi = __uint_as_float(w[e] & 0xFFFF0000u);
-              ss += static_cast<double>(lo * lo);
-              ss += static_cast<double>(hi * hi);
+              ss += __hiloint2double(static_cast<int>(__umulhi(__float_as_uint(lo * lo), 1u << 29) + 0x38000000u), 0);
+              ss += __hiloint2double(static_cast<int>(__umulhi(__float_as_uint(hi * hi), 1u << 29) + 0x38000000u), 0);
             }
           }
           if (row < p.M) {

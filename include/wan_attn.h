@@ -204,6 +204,26 @@ WAN_API int32_t wan_qk_norm_rope_stats(void* qkv, int64_t batch, int32_t F, int3
                                        float theta, const double* stats, void* stream);
 
 /*
+ * Sequence parallelism (the fourth NEXT item; Neuron page, "Context
+ * parallelism": each rank owns S/N tokens, and its queries must attend every
+ * key). Two calls make a rank's share of the path:
+ * wan_qk_norm_rope_shard: (1) on a buffer holding tokens [s0, s0 + s_local)
+ *   of every batch element's F x H x W grid ([batch][s_local][3*heads*128];
+ *   RoPE positions from the grid index s0 + i). 0 <= s0, s0 + s_local <= F*H*W.
+ * wan_self_attention_rows: (2) for query rows [q_row0, q_row0 + q_rows) of the
+ *   full packed buffer qkv ([batch][seq_len][3*heads*128], every key present,
+ *   e.g. after an all-gather of the normalised shards); out holds q_rows rows
+ *   per batch element ([batch][q_rows][heads*128]). 0 <= q_row0,
+ *   q_row0 + q_rows <= seq_len.
+ * The bits equal those of the unsharded calls for the same rows.
+ */
+WAN_API int32_t wan_qk_norm_rope_shard(void* qkv, int64_t batch, int32_t F, int32_t H, int32_t W, int64_t s0,
+                                       int64_t s_local, int32_t heads, int32_t head_dim, const void* gamma_q,
+                                       const void* gamma_k, float eps, float theta, void* stream);
+WAN_API int32_t wan_self_attention_rows(const void* qkv, void* out, int64_t batch, int64_t seq_len, int32_t heads,
+                                        int32_t head_dim, int64_t q_row0, int64_t q_rows, float scale, void* stream);
+
+/*
  * Synchronises `stream`, then reads and clears the Skip-Softmax counters
  * accumulated by wan_self_attention_sparse launches since the last read:
  * *group_tiles = (32-row group, key tile) pairs skipped, *products = 128-row

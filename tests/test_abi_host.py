@@ -39,7 +39,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings(lib):
-    assert lib.wan_abi_version() == 6
+    assert lib.wan_abi_version() == 7
     for code in range(11):
         assert lib.wan_status_string(code)
     assert lib.wan_status_string(99) == b"unknown status"
@@ -176,3 +176,14 @@ def test_linear_validates(lib):
     import torch
     if not torch.cuda.is_available():
         assert lib.wan_linear(FAKE, FAKE, far, 4, 256, 64, None, 0, None) == 6
+
+
+def test_sequence_shard_entry_points_validate(lib):
+    # wan_qk_norm_rope_shard(qkv, batch, F, H, W, s0, s_local, heads, head_dim, gq, gk, eps, theta)
+    assert lib.wan_qk_norm_rope_shard(FAKE, 1, 2, 2, 2, 4, 5, 1, 128, FAKE, FAKE, 1e-6, 1e4, None) == 3
+    assert lib.wan_qk_norm_rope_shard(FAKE, 1, 2, 2, 2, -1, 4, 1, 128, FAKE, FAKE, 1e-6, 1e4, None) == 3
+    assert lib.wan_qk_norm_rope_shard(None, 1, 2, 2, 2, 0, 4, 1, 128, FAKE, FAKE, 1e-6, 1e4, None) == 1
+    # wan_self_attention_rows(qkv, out, batch, S, heads, head_dim, q_row0, q_rows, scale)
+    assert lib.wan_self_attention_rows(FAKE, 2**40, 1, 8, 1, 128, 6, 3, 0.0, None) == 3
+    assert lib.wan_self_attention_rows(FAKE, 2**40, 1, 8, 1, 128, 0, 0, 0.0, None) == 3
+    assert lib.wan_self_attention_rows(FAKE, FAKE + 64, 1, 8, 1, 128, 0, 4, 0.0, None) == 9

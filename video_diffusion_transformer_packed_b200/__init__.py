@@ -20,7 +20,7 @@ from typing import Optional, Sequence
 
 __all__ = ["WanError", "load_library", "library_path", "qk_norm_rope", "self_attention",
            "self_attention_sparse", "skip_stats", "qkv_amax", "quantize_fp8", "self_attention_fp8",
-           "fp8_pitch", "linear", "qk_norm_rope_stats", "dit_attn", "dit_attn_host", "device_error", "selftest_wait_timeout", "HEAD_DIM", "EPS",
+           "fp8_pitch", "linear", "qk_norm_rope_stats", "qk_norm_rope_shard", "self_attention_rows", "dit_attn", "dit_attn_host", "device_error", "selftest_wait_timeout", "HEAD_DIM", "EPS",
            "THETA", "STATUS"]
 
 HEAD_DIM = 128
@@ -91,6 +91,10 @@ def load_library() -> ctypes.CDLL:
             lib.wan_linear.restype = I32
             lib.wan_qk_norm_rope_stats.argtypes = [P, I64, I32, I32, I32, I32, I32, P, P, F, F, P, P]
             lib.wan_qk_norm_rope_stats.restype = I32
+            lib.wan_qk_norm_rope_shard.argtypes = [P, I64, I32, I32, I32, I64, I64, I32, I32, P, P, F, F, P]
+            lib.wan_qk_norm_rope_shard.restype = I32
+            lib.wan_self_attention_rows.argtypes = [P, P, I64, I64, I32, I32, I64, I64, F, P]
+            lib.wan_self_attention_rows.restype = I32
             _lib = lib
     return _lib
 
@@ -289,6 +293,39 @@ def qk_norm_rope_stats(qkv, grid: Sequence[int], heads: int, gamma_q, gamma_k, s
                                                  eps, theta, stats.data_ptr(), _stream(stream)),
            "wan_qk_norm_rope_stats")
     return qkv
+
+
+def qk_norm_rope_shard(qkv_local, grid: Sequence[int], heads: int, s0: int, gamma_q, gamma_k, eps: float = EPS,
+                       theta: float = THETA, stream=None):
+    """qk_norm_rope on a sequence shard: qkv_local [B, s_local, 3*heads*128]
+    holds tokens [s0, s0 + s_local) of every batch element's grid."""
+    F, H, W = grid
+    B, S_l, d3 = qkv_local.shape
+    if d3 != 3 * heads * HEAD_DIM:
+        raise ValueError("qkv_local must be [B, s_local, 3*heads*128]")
+    _check_gamma(gamma_q, heads, "gamma_q")
+    _check_gamma(gamma_k, heads, "gamma_k")
+    _check(load_library().wan_qk_norm_rope_shard(_bf16_cuda(qkv_local, "qkv_local"), B, F, H, W, int(s0), S_l,
+                                                 heads, HEAD_DIM, _bf16_cuda(gamma_q, "gamma_q"),
+                                                 _bf16_cuda(gamma_k, "gamma_k"), eps, theta, _stream(stream)),
+           "wan_qk_norm_rope_shard")
+    return qkv_local
+
+
+def self_attention_rows(qkv, heads: int, q_row0: int, q_rows: int, out=None, scale: float = 0.0, stream=None):
+    """Attention of query rows [q_row0, q_row0 + q_rows) of the full packed
+    buffer against every key: out [B, q_rows, heads*128]."""
+    import torch
+    _check_packed(qkv, heads)
+    B, S, _ = qkv.shape
+    if out is None:
+        out = torch.empty((B, q_rows, heads * HEAD_DIM), dtype=torch.bfloat16, device=qkv.device)
+    if tuple(out.shape) != (B, q_rows, heads * HEAD_DIM):
+        raise ValueError("out must be [B, q_rows, heads*128]")
+    _check(load_library().wan_self_attention_rows(_bf16_cuda(qkv, "qkv"), _bf16_cuda(out, "out"), B, S, heads,
+                                                  HEAD_DIM, int(q_row0), int(q_rows), scale, _stream(stream)),
+           "wan_self_attention_rows")
+    return out
 
 
 def dit_attn(qkv, grid: Sequence[int], heads: int, gamma_q, gamma_k, out=None, eps: float = EPS,

@@ -11,7 +11,7 @@
 
 namespace {
 
-constexpr int32_t kAbiVersion = 6;
+constexpr int32_t kAbiVersion = 7;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -300,6 +300,46 @@ int32_t wan_qk_norm_rope_stats(void* qkv, int64_t batch, int32_t F, int32_t H, i
                                static_cast<cudaStream_t>(stream), stats) != cudaSuccess) {
     return WAN_ERR_LAUNCH;
   }
+  return WAN_OK;
+}
+
+int32_t wan_qk_norm_rope_shard(void* qkv, int64_t batch, int32_t F, int32_t H, int32_t W, int64_t s0,
+                               int64_t s_local, int32_t heads, int32_t head_dim, const void* gamma_q,
+                               const void* gamma_k, float eps, float theta, void* stream) {
+  int64_t S = 0;
+  WAN_TRY(check_heads(heads, head_dim));
+  WAN_TRY(check_grid(batch, F, H, W, heads, &S));
+  if (s0 < 0 || s_local < 1 || s0 + s_local > S) return WAN_ERR_SHAPE;
+  WAN_TRY(check_norm_args(qkv, gamma_q, gamma_k, eps, theta));
+  WAN_TRY(check_device());
+  (void)cudaGetLastError();
+  if (wan::launch_qk_norm_rope(qkv, batch, F, H, W, heads, gamma_q, gamma_k, eps, theta,
+                               static_cast<cudaStream_t>(stream), nullptr, s0, s_local) != cudaSuccess) {
+    return WAN_ERR_LAUNCH;
+  }
+  return WAN_OK;
+}
+
+int32_t wan_self_attention_rows(const void* qkv, void* out, int64_t batch, int64_t seq_len, int32_t heads,
+                                int32_t head_dim, int64_t q_row0, int64_t q_rows, float scale, void* stream) {
+  WAN_TRY(check_heads(heads, head_dim));
+  WAN_TRY(check_tokens(batch, seq_len, heads));
+  if (q_row0 < 0 || q_rows < 1 || q_row0 + q_rows > seq_len) return WAN_ERR_SHAPE;
+  if (!qkv || !out) return WAN_ERR_NULL;
+  if (!aligned16(qkv) || !aligned16(out)) return WAN_ERR_ALIGN;
+  if (!std::isfinite(scale)) return WAN_ERR_PARAM;
+  const uint64_t d = static_cast<uint64_t>(heads) * WAN_HEAD_DIM;
+  if (overlaps(qkv, static_cast<uint64_t>(batch) * seq_len * 3 * d * 2, out,
+               static_cast<uint64_t>(batch) * q_rows * d * 2)) {
+    return WAN_ERR_ALIAS;
+  }
+  WAN_TRY(check_device());
+  (void)cudaGetLastError();
+  wan::AttnPlan plan;
+  if (wan::plan_attn_fwd(qkv, out, batch, seq_len, heads, scale, &plan) != cudaSuccess) return WAN_ERR_LAUNCH;
+  plan.q_row0 = static_cast<int32_t>(q_row0);
+  plan.q_rows = static_cast<int32_t>(q_rows);
+  if (wan::launch_attn_fwd(plan, static_cast<cudaStream_t>(stream), false) != cudaSuccess) return WAN_ERR_LAUNCH;
   return WAN_OK;
 }
 

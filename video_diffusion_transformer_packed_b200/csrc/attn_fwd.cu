@@ -97,6 +97,7 @@ struct AttnParams {
   int32_t q_pairs;  // ceil(S / 256): CTAs per (batch, head)
   int32_t n_kv;     // ceil(S / 128)
   int32_t b0, h0, nh;  // this launch covers batches [b0, ...) and heads [h0, h0 + nh)
+  int32_t q_row0, q_rows;  // query rows [q_row0, q_row0 + q_rows); out holds q_rows rows per batch
   float skip_log2;     // Skip-Softmax: log2 of the threshold (used by the kSkip kernel only)
   float scale_log2; // scale * log2(e)
   uint64_t wait_ns; // limit of each pipeline wait
@@ -134,7 +135,7 @@ __device__ void run_producer(const CUtensorMap* tmap, const AttnParams& p, uint3
   for (int t = 0; t < 2; ++t) {
     for (int half = 0; half < 2; ++half) {
       tma_load_3d(smem + kOffQ + t * kTileBytes + half * kBoxBytes, tmap, bars.q_full(),
-                  xq + 64 * half, (2 * qp + t) * kBM, b);
+                  xq + 64 * half, p.q_row0 + (2 * qp + t) * kBM, b);
     }
   }
   bool ok = true;
@@ -334,7 +335,7 @@ __device__ void run_softmax(const AttnParams& p, Bars bars, volatile int* abort,
   float m_run = -INFINITY;  // running max, already in scaled log2 units
   float l_run = 0.f;
   float m_true = -INFINITY;  // exact running max (Skip-Softmax decisions)
-  const bool row_valid = (2 * qp + t) * kBM + quarter * 32 + lane < p.S;
+  const bool row_valid = (2 * qp + t) * kBM + quarter * 32 + lane < p.q_rows;
   uint32_t n_skipped = 0;
   bool ok = true;
 
@@ -456,14 +457,14 @@ __device__ void run_softmax(const AttnParams& p, Bars bars, volatile int* abort,
   }
   tc_fence_after();
   const float inv_l = 1.f / l_run;
-  const int row = (2 * qp + t) * kBM + quarter * 32 + lane;
-  uint16_t* dst = p.out + (static_cast<int64_t>(b) * p.S + row) * p.D + h * kHD;
+  const int row = (2 * qp + t) * kBM + quarter * 32 + lane;  // within this launch's query rows
+  uint16_t* dst = p.out + (static_cast<int64_t>(b) * p.q_rows + row) * p.D + h * kHD;
 #pragma unroll 1
   for (int c = 0; c < 4; ++c) {
     uint32_t o[32];
     tmem_ld32(tO + 32 * c, o);
     tmem_wait_ld();
-    if (row < p.S) {
+    if (row < p.q_rows) {
       uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
 #pragma unroll
       for (int v = 0; v < 4; ++v) {
@@ -612,6 +613,8 @@ cudaError_t plan_attn_fwd(const void* qkv, void* out, int64_t batch, int64_t seq
   const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(kHD));
   plan->scale_log2 = sc * 1.4426950408889634f;
   plan->skip_threshold = 0.f;
+  plan->q_row0 = 0;
+  plan->q_rows = S;
   plan->b0 = 0;
   plan->nb = static_cast<int32_t>(batch);
   plan->h0 = 0;
@@ -626,11 +629,13 @@ cudaError_t launch_attn_fwd(const AttnPlan& plan, cudaStream_t stream, bool pdl,
   p.S = plan.S;
   p.heads = plan.heads;
   p.D = plan.D;
-  p.q_pairs = plan.q_pairs;
   p.n_kv = plan.n_kv;
   p.b0 = plan.b0;
   p.h0 = plan.h0;
   p.nh = plan.nh;
+  p.q_row0 = plan.q_row0;
+  p.q_rows = plan.q_rows;
+  p.q_pairs = (plan.q_rows + 2 * kBM - 1) / (2 * kBM);
   p.scale_log2 = plan.scale_log2;
   p.skip_log2 = plan.skip_threshold > 0.f ? log2f(plan.skip_threshold) : -INFINITY;
   p.wait_ns = wait_ns;
@@ -639,8 +644,9 @@ cudaError_t launch_attn_fwd(const AttnPlan& plan, cudaStream_t stream, bool pdl,
   memcpy(&tmap, plan.tmap, sizeof(tmap));
 
   cudaLaunchConfig_t cfg = {};
-  const int64_t grid = static_cast<int64_t>(plan.nb) * plan.nh * plan.q_pairs;
+  const int64_t grid = static_cast<int64_t>(plan.nb) * plan.nh * p.q_pairs;
   if (plan.nb < 1 || plan.nh < 1 || plan.h0 < 0 || plan.b0 < 0 || plan.h0 + plan.nh > plan.heads ||
+      plan.q_row0 < 0 || plan.q_rows < 1 || static_cast<int64_t>(plan.q_row0) + plan.q_rows > plan.S ||
       grid > INT32_MAX) {
     return cudaErrorInvalidValue;
   }

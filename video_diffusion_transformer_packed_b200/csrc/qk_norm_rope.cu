@@ -69,7 +69,8 @@ struct NormRopeParams {
   const uint16_t* gamma_q;
   const uint16_t* gamma_k;
   int64_t tokens;        // batch * S
-  int32_t S, H, W;
+  int32_t S, H, W;       // S: tokens per batch element in this buffer
+  int32_t s0;            // grid index of the buffer's first token (a sequence shard starts past 0)
   int32_t D;             // heads * 128
   int32_t nvec;          // D / 8 sixteen-byte vectors per row
   int32_t stages;        // ring depth
@@ -269,7 +270,7 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const __grid_
   const int step_mod = static_cast<int>(step % p.S);
   int s_next = static_cast<int>(blockIdx.x % p.S);
   const int my_pr = tid >> 2;  // the pair whose rotation this thread computes (every 4th thread)
-  if ((tid & 3) == 0) rotation(p, s_next, my_pr, tail.rot[0]);
+  if ((tid & 3) == 0) rotation(p, s_next + p.s0, my_pr, tail.rot[0]);
   s_next += step_mod;
   if (s_next >= p.S) s_next -= p.S;
   __syncthreads();
@@ -287,7 +288,7 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const __grid_
     }
     // The next token's rotations, ahead of time (they do not depend on the data).
     const int rnext = rbuf == 2 ? 0 : rbuf + 1;
-    if ((tid & 3) == 0 && tok + step < p.tokens) rotation(p, s_next, my_pr, tail.rot[rnext]);
+    if ((tid & 3) == 0 && tok + step < p.tokens) rotation(p, s_next + p.s0, my_pr, tail.rot[rnext]);
     if (!mbar_wait(smem_u32(&tail.full[stage]), parity, nullptr, kWaitLimitNs)) {
       tail.abort = 1;
       atomicOr(&g_norm_error_word, 1);
@@ -451,12 +452,14 @@ cudaError_t launch_vpt_dispatch(int vpt, const NormRopeParams& p, uint32_t smem_
 
 cudaError_t launch_qk_norm_rope(void* qkv, int64_t batch, int32_t F, int32_t H, int32_t W,
                                 int32_t heads, const void* gamma_q, const void* gamma_k, float eps,
-                                float theta, cudaStream_t stream, const double* stats) {
+                                float theta, cudaStream_t stream, const double* stats, int64_t s0,
+                                int64_t s_local) {
   NormRopeParams p;
   p.qkv = static_cast<uint16_t*>(qkv);
   p.gamma_q = static_cast<const uint16_t*>(gamma_q);
   p.gamma_k = static_cast<const uint16_t*>(gamma_k);
-  p.S = F * H * W;
+  p.S = s_local > 0 ? static_cast<int32_t>(s_local) : F * H * W;
+  p.s0 = static_cast<int32_t>(s0);
   p.H = H;
   p.W = W;
   p.D = heads * kHeadDim;

@@ -12,9 +12,12 @@ namespace wan {
 // With `stats` (the QKV projection's per-256-column sums of squares of the
 // same buffer, [batch*S][2*heads*128/256] fp64, see launch_gemm_bf16) the kernel
 // takes each row's sum from them instead of reducing it.
+// With s_local > 0 the buffer holds a sequence shard: tokens [s0, s0 + s_local)
+// of every batch element's F x H x W grid (positions from the grid index).
 cudaError_t launch_qk_norm_rope(void* qkv, int64_t batch, int32_t F, int32_t H, int32_t W,
                                 int32_t heads, const void* gamma_q, const void* gamma_k, float eps,
-                                float theta, cudaStream_t stream, const double* stats = nullptr);
+                                float theta, cudaStream_t stream, const double* stats = nullptr,
+                                int64_t s0 = 0, int64_t s_local = 0);
 
 // Everything the attention launch needs, prepared before anything is
 // launched (tensor-map encoding can fail; a launch after a successful plan
@@ -30,6 +33,9 @@ struct AttnPlan {
   int32_t b0, nb, h0, nh;
   // Skip-Softmax threshold (0 = dense; plan_attn_fwd sets 0).
   float skip_threshold;
+  // Query rows [q_row0, q_row0 + q_rows) of every batch element attend all S
+  // keys; out holds q_rows rows per batch element (plan_attn_fwd: 0 and S).
+  int32_t q_row0, q_rows;
 };
 
 cudaError_t plan_attn_fwd(const void* qkv, void* out, int64_t batch, int64_t seq_len,

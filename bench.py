@@ -336,20 +336,25 @@ def run_ours(args):
     # ---- end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
-        # wan_dit_attn_host: the input arrives from pinned host memory and the
-        # output returns to it, copies overlapped with the kernels inside the
-        # library; every byte of both crosses PCIe inside the timed region.
-        qkv = bufs[0]
-        out_pinned = torch.empty((w.batch, w.seq_len, w.dim), dtype=torch.bfloat16).pin_memory()
+        # wan_dit_attn_host: each step's input arrives from pinned host memory
+        # and its output returns to pinned host memory, the copies overlapped
+        # with the kernels inside the library; every byte of both crosses PCIe
+        # inside the timed region. Two device buffer sets alternate between
+        # steps, so a step's input transfer also overlaps the previous step's
+        # kernels (WAN_HOST_OVERLAP_INPUT).
+        sets = [(bufs[0], out), (bufs[1] if nbuf > 1 else torch.empty_like(bufs[0]), torch.empty_like(out))]
+        outs_pinned = [torch.empty((w.batch, w.seq_len, w.dim), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
         h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         for k in range(args.warmup + args.steps):
             if k == args.warmup:
                 stream.synchronize()
                 h0.record(stream)
-            wan.dit_attn_host(qkv_pinned, w.grid, w.heads, gq, gk, out_host=out_pinned, qkv_dev=qkv,
-                              out_dev=out, stream=stream)
+            qd, od = sets[k % 2]
+            wan.dit_attn_host(qkv_pinned, w.grid, w.heads, gq, gk, out_host=outs_pinned[k % 2], qkv_dev=qd,
+                              out_dev=od, overlap_input=True, stream=stream)
         h1.record(stream)
         stream.synchronize()
+        qkv = bufs[0]
         e2e_ms = max_over_ranks(h0.elapsed_time(h1), dev, pg)
         e2e = {"value": job_throughput(world, w.attn_flop, args.steps, e2e_ms), "unit": "TFLOP/s",
                "h2d_bytes_per_step": qkv.numel() * 2, "d2h_bytes_per_step": out.numel() * 2,

@@ -77,6 +77,13 @@ typedef enum {
                                      is not memory of the current device */
 } wan_status;
 
+/* wan_dit_attn_host flag: the copies into qkv_dev start without waiting for
+ * earlier work on `stream`. The caller guarantees that no earlier work still
+ * uses qkv_dev or out_dev (e.g. it alternates two sets between consecutive
+ * calls), so that one call's input transfer overlaps the previous call's
+ * kernels. */
+#define WAN_HOST_OVERLAP_INPUT 1
+
 /* Default head-chunk size of wan_dit_attn_host's pipeline. */
 #define WAN_HOST_HEADS_PER_CHUNK 8
 /* Largest number of (batch element, head chunk) pieces one wan_dit_attn_host
@@ -262,9 +269,11 @@ WAN_API int32_t wan_dit_attn(void* qkv, void* out, int64_t batch, int32_t F, int
  *           must not overlap qkv_dev.
  * heads_per_chunk  1..heads, or 0 for WAN_HOST_HEADS_PER_CHUNK (capped at
  *           heads); batch * ceil(heads/heads_per_chunk) <= WAN_HOST_MAX_PIECES.
+ * flags     0 or WAN_HOST_OVERLAP_INPUT.
  * Other arguments as for wan_dit_attn. Device pointers 16-byte aligned.
  * Execution: asynchronous and ordered on `stream`: the copies into qkv_dev
- * start after the work enqueued on `stream` before this call, and work
+ * start after the work enqueued on `stream` before this call (unless
+ * WAN_HOST_OVERLAP_INPUT), and work
  * enqueued on `stream` after it runs once out_host is written (synchronise
  * `stream` before reading out_host on the host). The library keeps two
  * internal streams per device for the copies; concurrent calls on one device
@@ -279,7 +288,7 @@ WAN_API int32_t wan_dit_attn_host(const void* qkv_host, void* out_host, void* qk
                                   int64_t batch, int32_t F, int32_t H, int32_t W, int32_t heads,
                                   int32_t head_dim, const void* gamma_q, const void* gamma_k,
                                   float eps, float theta, float scale, int32_t heads_per_chunk,
-                                  void* stream);
+                                  int32_t flags, void* stream);
 
 /*
  * Synchronises `stream`, then reads and clears the device-side error words

@@ -39,7 +39,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings(lib):
-    assert lib.wan_abi_version() == 7
+    assert lib.wan_abi_version() == 8
     for code in range(11):
         assert lib.wan_status_string(code)
     assert lib.wan_status_string(99) == b"unknown status"
@@ -114,8 +114,9 @@ def test_host_pipeline_validates_before_touching_memory(lib):
         names = ["qh", "oh", "qd", "od", "b", "F", "H", "W", "heads", "hd", "gq", "gk", "eps", "theta",
                  "scale", "hc"]
         for k, v in kw.items():
-            a[names.index(k)] = v
-        return lib.wan_dit_attn_host(*a, None)
+            if k != "flags":
+                a[names.index(k)] = v
+        return lib.wan_dit_attn_host(*a, kw.get("flags", 0), None) if "flags" in kw else lib.wan_dit_attn_host(*a, 0, None)
 
     assert call(qh=None) == 1
     assert call(oh=None) == 1
@@ -127,6 +128,7 @@ def test_host_pipeline_validates_before_touching_memory(lib):
     assert call(od=FAKE + 64) == 9  # out_dev overlaps qkv_dev
     assert call(hc=-1) == 5
     assert call(hc=5) == 5  # more than heads
+    assert call(flags=2) == 5  # unknown flag
     assert call(b=5000, hc=1, od=2**40) == 3  # more pieces than the pipeline takes
     import torch
     if not torch.cuda.is_available():

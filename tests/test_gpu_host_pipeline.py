@@ -104,7 +104,7 @@ def test_host_pipeline_refuses_pageable_or_foreign_memory():
     out_d = torch.empty((1, w.seq_len, w.dim), dtype=torch.bfloat16, device="cuda")
     out_pageable = torch.empty((1, w.seq_len, w.dim), dtype=torch.bfloat16)
     args = [qkv.data_ptr(), out_pageable.data_ptr(), qkv_d.data_ptr(), out_d.data_ptr(), 1, *w.grid,
-            w.heads, 128, gq.data_ptr(), gk.data_ptr(), wi.EPS, wi.THETA, 0.0, 0, None]
+            w.heads, 128, gq.data_ptr(), gk.data_ptr(), wi.EPS, wi.THETA, 0.0, 0, 0, None]
     assert lib.wan_dit_attn_host(*args) == 10  # pageable host memory
     qkv_h, out_h = _pinned(qkv), _pinned(out_pageable)
     args[0], args[1] = qkv_h.data_ptr(), out_h.data_ptr()
@@ -113,3 +113,25 @@ def test_host_pipeline_refuses_pageable_or_foreign_memory():
     args[2] = qkv_d.data_ptr()
     assert lib.wan_dit_attn_host(*args) == 0
     torch.cuda.synchronize()
+
+
+def test_overlapped_calls_with_alternating_buffers():
+    """WAN_HOST_OVERLAP_INPUT with two alternating device buffer sets on one
+    stream: every call's output equals the device path's."""
+    w = wi.Workload("case", 2, (2, 10, 13), 7)
+    gq_h, gk_h = wi.gammas(w.heads)
+    gq, gk = gq_h.cuda(), gk_h.cuda()
+    s = torch.cuda.Stream()
+    sets = [(torch.empty((w.batch, w.seq_len, 3 * w.dim), dtype=torch.bfloat16, device="cuda"),
+             torch.empty((w.batch, w.seq_len, w.dim), dtype=torch.bfloat16, device="cuda")) for _ in range(2)]
+    outs, refs = [], []
+    for k, seed in enumerate((31, 32, 33, 34)):
+        qkv = wi.packed_qkv(w.batch, w.seq_len, w.heads, seed=seed)
+        _, ref = _device_reference(qkv, w, gq, gk)
+        refs.append(ref.cpu())
+        qd, od = sets[k % 2]
+        outs.append(wan.dit_attn_host(_pinned(qkv), w.grid, w.heads, gq, gk, qkv_dev=qd, out_dev=od,
+                                      heads_per_chunk=3, overlap_input=True, stream=s))
+    s.synchronize()
+    for o, r in zip(outs, refs):
+        assert torch.equal(o.view(torch.int16), r.view(torch.int16))

@@ -75,7 +75,7 @@ def load_library() -> ctypes.CDLL:
             lib.wan_selftest_wait_timeout.argtypes = [P, P, I64, I64, I32, I32, I64, P]
             lib.wan_selftest_wait_timeout.restype = I32
             lib.wan_dit_attn_host.argtypes = [P, P, P, P, I64, I32, I32, I32, I32, I32, P, P, F, F, F,
-                                              I32, P]
+                                              I32, I32, P]
             lib.wan_dit_attn_host.restype = I32
             lib.wan_self_attention_sparse.argtypes = [P, P, I64, I64, I32, I32, F, F, P]
             lib.wan_self_attention_sparse.restype = I32
@@ -356,13 +356,14 @@ def _bf16_pinned(t, name: str) -> int:
 
 def dit_attn_host(qkv_host, grid: Sequence[int], heads: int, gamma_q, gamma_k, out_host=None,
                   qkv_dev=None, out_dev=None, heads_per_chunk: int = 0, eps: float = EPS,
-                  theta: float = THETA, scale: float = 0.0, stream=None):
+                  theta: float = THETA, scale: float = 0.0, overlap_input: bool = False, stream=None):
     """The step for packed qkv in page-locked host memory: host->device copies,
     qk_norm_rope, self_attention and the device->host copy of the output,
     overlapped chunk by chunk inside the library. qkv_dev / out_dev are the
     device buffers it runs through (allocated on the current device when not
     given); qkv_host is only read. Asynchronous on `stream`: synchronise it
-    before reading out_host."""
+    before reading out_host. overlap_input: the input transfer does not wait
+    for earlier work on `stream` (the caller alternates device buffer sets)."""
     import torch
     F, H, W = grid
     _check_packed(qkv_host, heads, grid)
@@ -386,7 +387,8 @@ def dit_attn_host(qkv_host, grid: Sequence[int], heads: int, gamma_q, gamma_k, o
                                             _bf16_cuda(qkv_dev, "qkv_dev"), _bf16_cuda(out_dev, "out_dev"),
                                             B, F, H, W, heads, HEAD_DIM, _bf16_cuda(gamma_q, "gamma_q"),
                                             _bf16_cuda(gamma_k, "gamma_k"), eps, theta, scale,
-                                            int(heads_per_chunk), _stream(stream)), "wan_dit_attn_host")
+                                            int(heads_per_chunk), 1 if overlap_input else 0, _stream(stream)),
+           "wan_dit_attn_host")
     return out_host
 
 

@@ -11,7 +11,7 @@
 
 namespace {
 
-constexpr int32_t kAbiVersion = 7;
+constexpr int32_t kAbiVersion = 8;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -381,7 +381,7 @@ int32_t wan_dit_attn(void* qkv, void* out, int64_t batch, int32_t F, int32_t H, 
 int32_t wan_dit_attn_host(const void* qkv_host, void* out_host, void* qkv_dev, void* out_dev,
                           int64_t batch, int32_t F, int32_t H, int32_t W, int32_t heads,
                           int32_t head_dim, const void* gamma_q, const void* gamma_k, float eps,
-                          float theta, float scale, int32_t heads_per_chunk, void* stream) {
+                          float theta, float scale, int32_t heads_per_chunk, int32_t flags, void* stream) {
   int64_t S = 0;
   WAN_TRY(check_heads(heads, head_dim));
   WAN_TRY(check_grid(batch, F, H, W, heads, &S));
@@ -389,6 +389,7 @@ int32_t wan_dit_attn_host(const void* qkv_host, void* out_host, void* qkv_dev, v
   WAN_TRY(check_norm_args(qkv_dev, gamma_q, gamma_k, eps, theta));
   WAN_TRY(check_attn_args(qkv_dev, out_dev, batch, S, heads, scale));
   if (heads_per_chunk < 0 || heads_per_chunk > heads) return WAN_ERR_PARAM;
+  if (flags & ~WAN_HOST_OVERLAP_INPUT) return WAN_ERR_PARAM;
   const int32_t hc = heads_per_chunk > 0 ? heads_per_chunk
                                          : (heads < WAN_HOST_HEADS_PER_CHUNK ? heads : WAN_HOST_HEADS_PER_CHUNK);
   if (batch * ((heads + hc - 1) / hc) > WAN_HOST_MAX_PIECES) return WAN_ERR_SHAPE;
@@ -412,6 +413,7 @@ int32_t wan_dit_attn_host(const void* qkv_host, void* out_host, void* qkv_dev, v
   step.eps = eps;
   step.theta = theta;
   step.scale = scale;
+  step.overlap_input = (flags & WAN_HOST_OVERLAP_INPUT) != 0;
   if (wan::enqueue_dit_attn_host(step, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
     return WAN_ERR_LAUNCH;
   }

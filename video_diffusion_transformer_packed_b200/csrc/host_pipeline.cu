@@ -89,9 +89,13 @@ cudaError_t enqueue_dit_attn_host(const HostStep& a, cudaStream_t user) {
   auto ev = [&]() { return q.events[next++]; };
   const cudaEvent_t ev_start = ev();
   // Copies must not overwrite the device buffers before earlier work on the
-  // caller's stream is done with them.
-  WAN_CUDA_TRY(cudaEventRecord(ev_start, user));
-  WAN_CUDA_TRY(cudaStreamWaitEvent(q.h2d, ev_start, 0));
+  // caller's stream is done with them -- unless the caller vouches that no
+  // earlier work uses these buffers (it alternates sets), in which case this
+  // call's transfer overlaps the previous call's kernels.
+  if (!a.overlap_input) {
+    WAN_CUDA_TRY(cudaEventRecord(ev_start, user));
+    WAN_CUDA_TRY(cudaStreamWaitEvent(q.h2d, ev_start, 0));
+  }
 
   auto* qkv_h = static_cast<const unsigned char*>(a.qkv_host);
   auto* qkv_d = static_cast<unsigned char*>(a.qkv_dev);

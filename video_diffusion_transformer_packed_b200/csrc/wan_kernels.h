@@ -63,6 +63,7 @@ struct HostStep {
   const void* gamma_q;
   const void* gamma_k;
   float eps, theta, scale;
+  bool overlap_input;  // copies in do not wait for earlier work on the stream
 };
 cudaError_t enqueue_dit_attn_host(const HostStep& step, cudaStream_t stream);
 

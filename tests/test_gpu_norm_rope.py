@@ -78,6 +78,23 @@ def test_large_positions_on_720p_axes():
     check_full(qkv, grid, heads, gq, gk)
 
 
+@pytest.mark.parametrize("batch,grid", [
+    (1, (4, 60, 150)),   # columns past 64 and 128, rows past the token range of a CTA
+    (2, (130, 2, 70)),   # frames past 128, a batch boundary inside CTAs' ranges
+    (3, (5, 97, 31)),    # rows past 64, odd sizes
+])
+def test_rotation_carried_across_long_axes(batch, grid):
+    """Tens of thousands of tokens at one head: every CTA walks many
+    consecutive tokens, so the kernel's step-by-step rotation update, its
+    fresh evaluation at wraps, jumps and every 64th position, and the batch
+    boundary all run; every element is checked."""
+    heads = 1
+    w = wi.Workload("t", batch, grid, heads)
+    qkv = wi.packed_qkv(batch, w.seq_len, heads, seed=sum(grid))
+    gq, gk = wi.gammas(heads, 15, 16)
+    check_full(qkv, grid, heads, gq, gk)
+
+
 @pytest.mark.parametrize("idx", [1, 2, 3, 4])
 def test_full_size_workloads_sampled_tokens(idx):
     w = wi.WORKLOADS[idx]

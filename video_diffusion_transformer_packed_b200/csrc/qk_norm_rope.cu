@@ -10,7 +10,8 @@
 // with head dims [0,44) on the frame axis, [44,86) on rows, [86,128) on columns.
 //
 // Design: the op is HBM-bound (read + write of Q and K once: 8*D bytes per
-// token, V untouched). A persistent grid (a few CTAs per SM) walks the tokens.
+// token, V untouched). A persistent grid (a few CTAs per SM) walks the
+// tokens, each CTA a contiguous range of them.
 // A token's Q and K rows are contiguous in the packed buffer, so one bulk
 // copy (cp.async.bulk, the untiled TMA) stages both into a shared-memory
 // ring several tokens ahead of the threads that consume them; the reads of
@@ -30,10 +31,13 @@
 //    v_hi = fl(x*g*r_hi), and recomputed exactly (sign of x*g*r - midpoint,
 //    with two FMAs) for the rare threads whose v_hi lies within 2 fp32 ulps
 //    of a bf16 rounding midpoint;
-//  - cos/sin from one fp64 sincos per thread (shared through shared memory),
-//    split as a 16-significant-bit head plus a float tail: the products of
-//    the 8-bit y with the heads are exact in fp32, so the rotation's only
-//    rounding is in the final sums.
+//  - cos/sin in fp64, one pair per thread of the first two warps, carried
+//    from token to token by the angle-addition formulas (a CTA's tokens are
+//    consecutive, so a pair's position mostly stays or steps by one) with a
+//    fresh sincospi at every jump; shared through shared memory, split as a
+//    16-significant-bit head plus a float tail: the products of the 8-bit y
+//    with the heads are exact in fp32, so the rotation's only rounding is in
+//    the final sums.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -85,6 +89,20 @@ struct NormRopeParams {
   double freq_pi[kPairs];  // per pair of a head: theta^(-2j/d_axis) / pi
 };
 
+// Cos/sin of the pairs' rotation angles, kept in shared memory from one
+// token to the next (by the thread that owns the pair). A CTA walks a
+// contiguous range of tokens, so a pair's axis position (frame, row or
+// column of the token) mostly stays or grows by one: growing by one turns the
+// angle by the pair's frequency (the angle-addition formulas in fp64, four
+// multiply-adds); anything else -- the first token, a wrap to 0, a jump at a
+// batch boundary, and every 64th position to bound the recurrence's rounding
+// drift -- is one fp64 sincospi.
+struct PairRotations {
+  double2 cs[kPairs];    // (cos, sin) of pos * freq
+  double2 step[kPairs];  // (cos, sin) of freq
+  int pos[kPairs];       // the axis position cs belongs to; -1: none yet
+};
+
 // Shared-memory layout behind the ring (offsets from the ring's end).
 struct alignas(16) NormSmemTail {
   uint64_t full[kMaxStages];
@@ -95,6 +113,7 @@ struct alignas(16) NormSmemTail {
   // tails. A warp reads the 16 entries of one (h, j): contiguous, no bank
   // conflicts. The table of iteration i+1 is written during iteration i.
   float4 rot[3][2][3][16];
+  PairRotations rs;
   int abort;
 };
 
@@ -141,18 +160,45 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
       : "memory");
 }
 
-// Rotation operands of pair `pr` for sequence index s (one fp64 sincos):
-// cos/sin split into a 16-significant-bit head and a float tail, written into
-// its lane of the two-pair table entry.
-__device__ __forceinline__ void rotation(const NormRopeParams& p, int s, int pr, float4 (&t)[2][3][16]) {
-  const int q = s / p.W;  // frame * H + row
-  const int pos = pr < kRowAxisPair0 ? q / p.H : (pr < kColAxisPair0 ? q - (q / p.H) * p.H : s - q * p.W);
-  double sd, cd;
-  sincospi(static_cast<double>(pos) * p.freq_pi[pr], &sd, &cd);  // angle = pos * freq
-  const float ch = __uint_as_float(__float_as_uint(static_cast<float>(cd)) & 0xFFFFFF00u);
-  const float sh = __uint_as_float(__float_as_uint(static_cast<float>(sd)) & 0xFFFFFF00u);
-  const float cl = static_cast<float>(cd - static_cast<double>(ch));
-  const float sl = static_cast<float>(sd - static_cast<double>(sh));
+// Grid coordinates (frame, row, column) of sequence index s_glob.
+struct GridPos {
+  int f, r, c;
+};
+__device__ __forceinline__ GridPos grid_pos(const NormRopeParams& p, int s_glob) {
+  const int q = s_glob / p.W;  // frame * H + row
+  GridPos g;
+  g.f = q / p.H;
+  g.r = q - g.f * p.H;
+  g.c = s_glob - q * p.W;
+  return g;
+}
+
+// Moves pair pr's rotation to the grid position g and returns its (cos, sin).
+__device__ __forceinline__ double2 rotation_move(const NormRopeParams& p, PairRotations& rs, int pr,
+                                                 const GridPos& g) {
+  const int pos = pr < kRowAxisPair0 ? g.f : (pr < kColAxisPair0 ? g.r : g.c);
+  const int old = rs.pos[pr];
+  double2 cs = rs.cs[pr];
+  if (pos == old) return cs;
+  if (pos == old + 1 && (pos & 63) != 0) {
+    const double2 st = rs.step[pr];
+    cs = make_double2(fma(cs.x, st.x, -cs.y * st.y), fma(cs.y, st.x, cs.x * st.y));
+  } else {
+    sincospi(static_cast<double>(pos) * p.freq_pi[pr], &cs.y, &cs.x);  // angle = pos * freq
+  }
+  rs.cs[pr] = cs;
+  rs.pos[pr] = pos;
+  return cs;
+}
+
+// The rotation operands of pair `pr`: cos/sin split into a 16-significant-bit
+// head and a float tail, written into the pair's lane of the two-pair table
+// entry.
+__device__ __forceinline__ void rotation_write(double2 cs, int pr, float4 (&t)[2][3][16]) {
+  const float ch = __uint_as_float(__float_as_uint(static_cast<float>(cs.x)) & 0xFFFFFF00u);
+  const float sh = __uint_as_float(__float_as_uint(static_cast<float>(cs.y)) & 0xFFFFFF00u);
+  const float cl = static_cast<float>(cs.x - static_cast<double>(ch));
+  const float sl = static_cast<float>(cs.y - static_cast<double>(sh));
   const int g = pr >> 2, h = (pr >> 1) & 1, side = pr & 1;
   float* t0 = reinterpret_cast<float*>(&t[h][0][g]);
   float* t1 = reinterpret_cast<float*>(&t[h][1][g]);
@@ -242,7 +288,11 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const __grid_
   const int warp = tid >> 5;
   const int which = warp >> 2;  // 0: Q, 1: K
   const int u = tid & (kRowThreads - 1);
-  const int64_t step = gridDim.x;
+  // This CTA's tokens: a contiguous range, the remainder spread one token
+  // each over the first CTAs.
+  const int64_t per_cta = p.tokens / gridDim.x, extra = p.tokens % gridDim.x;
+  const int64_t t_begin = blockIdx.x * per_cta + (blockIdx.x < extra ? blockIdx.x : extra);
+  const int64_t t_end = t_begin + per_cta + (blockIdx.x < extra ? 1 : 0);
 
   if (tid == 0) {
     for (int s = 0; s < p.stages; ++s) mbar_init(smem_u32(&tail.full[s]), 1);
@@ -253,8 +303,8 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const __grid_
   int64_t n_issued = 0;  // copies started (thread 0 only): iterations 0 .. n_issued-1
   if (tid == 0) {
     for (int s = 0; s < p.stages; ++s) {
-      const int64_t tok = blockIdx.x + s * step;
-      if (tok < p.tokens) {
+      const int64_t tok = t_begin + s;
+      if (tok < t_end) {
         const uint32_t bar = smem_u32(&tail.full[s]);
         mbar_arrive_expect_tx(bar, p.stage_bytes);
         bulk_load(ring + s * p.stage_bytes, p.qkv + tok * 3 * static_cast<int64_t>(p.D), p.stage_bytes, bar);
@@ -265,20 +315,35 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const __grid_
 
   const uint16_t* g = which ? p.gamma_k : p.gamma_q;
 
-  // Sequence index of the current token and of the next one, kept
-  // incrementally (no 64-bit division in the loop).
-  const int step_mod = static_cast<int>(step % p.S);
-  int s_next = static_cast<int>(blockIdx.x % p.S);
-  const int my_pr = tid >> 2;  // the pair whose rotation this thread computes (every 4th thread)
-  if ((tid & 3) == 0) rotation(p, s_next + p.s0, my_pr, tail.rot[0]);
-  s_next += step_mod;
-  if (s_next >= p.S) s_next -= p.S;
+  // Threads 0-63 own the rotations of pairs 0-63 and keep them, with the
+  // sequence index and grid position of the next token, from one token to
+  // the next (no division in the loop but at a batch boundary).
+  const bool rot_thread = tid < kPairs;
+  int s_next = static_cast<int>(t_begin % p.S);
+  GridPos gp_next = grid_pos(p, s_next + p.s0);
+  if (rot_thread) {
+    double2 st;
+    sincospi(p.freq_pi[tid], &st.y, &st.x);
+    tail.rs.step[tid] = st;
+    tail.rs.pos[tid] = -1;
+    rotation_write(rotation_move(p, tail.rs, tid, gp_next), tid, tail.rot[0]);
+    if (++s_next == p.S) {
+      s_next = 0;
+      gp_next = grid_pos(p, p.s0);
+    } else if (++gp_next.c == p.W) {
+      gp_next.c = 0;
+      if (++gp_next.r == p.H) {
+        gp_next.r = 0;
+        ++gp_next.f;
+      }
+    }
+  }
   __syncthreads();
 
   int stage = 0, rbuf = 0;
   uint32_t parity = 0;
   int64_t i = 0;
-  for (int64_t tok = blockIdx.x; tok < p.tokens; tok += step, ++i) {
+  for (int64_t tok = t_begin; tok < t_end; ++tok, ++i) {
     const int buf = static_cast<int>(i & 1);
     // With precomputed statistics, lane j of each warp fetches the row's j-th
     // partial sum now; the load's latency hides behind the ring wait.
@@ -288,7 +353,19 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const __grid_
     }
     // The next token's rotations, ahead of time (they do not depend on the data).
     const int rnext = rbuf == 2 ? 0 : rbuf + 1;
-    if ((tid & 3) == 0 && tok + step < p.tokens) rotation(p, s_next + p.s0, my_pr, tail.rot[rnext]);
+    if (rot_thread && tok + 1 < t_end) {
+      rotation_write(rotation_move(p, tail.rs, tid, gp_next), tid, tail.rot[rnext]);
+      if (++s_next == p.S) {
+        s_next = 0;
+        gp_next = grid_pos(p, p.s0);
+      } else if (++gp_next.c == p.W) {
+        gp_next.c = 0;
+        if (++gp_next.r == p.H) {
+          gp_next.r = 0;
+          ++gp_next.f;
+        }
+      }
+    }
     if (!mbar_wait(smem_u32(&tail.full[stage]), parity, nullptr, kWaitLimitNs)) {
       tail.abort = 1;
       atomicOr(&g_norm_error_word, 1);
@@ -321,8 +398,8 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const __grid_
     if (tail.abort) break;
 
     if (tid == 0) {
-      const int64_t next = tok + p.stages * step;
-      if (next < p.tokens) {
+      const int64_t next = tok + p.stages;
+      if (next < t_end) {
         const uint32_t bar = smem_u32(&tail.full[stage]);
         mbar_arrive_expect_tx(bar, p.stage_bytes);
         bulk_load(ring + stage * p.stage_bytes, p.qkv + next * 3 * static_cast<int64_t>(p.D),
@@ -389,8 +466,6 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const __grid_
       if (vi < p.nvec) st_v4(x + 8 * vi, make_uint4(y[k][0], y[k][1], y[k][2], y[k][3]));
     }
     rbuf = rnext;
-    s_next += step_mod;
-    if (s_next >= p.S) s_next -= p.S;
     if (++stage == p.stages) {
       stage = 0;
       parity ^= 1u;

@@ -573,20 +573,18 @@ cudaError_t plan_attn_fwd(const void* qkv, void* out, int64_t batch, int64_t seq
   auto encode = get_encode_fn();
   if (!encode) return cudaErrorNotSupported;
 
-  static std::once_flag attr_once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(attr_once, [] {
+  static PerDeviceOnce setup;
+  const cudaError_t attr_err = setup.run([](int) {
     // The register split inside the kernel is only safe when the compiled
     // kernel launches with exactly kLaunchRegs registers per thread.
     for (auto kernel : {attn_fwd_kernel<false>, attn_fwd_kernel<true>}) {
       cudaFuncAttributes fa;
-      attr_err = cudaFuncGetAttributes(&fa, kernel);
-      if (attr_err == cudaSuccess && fa.numRegs != kLaunchRegs) attr_err = cudaErrorInvalidKernelImage;
-      if (attr_err == cudaSuccess) {
-        attr_err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-      }
-      if (attr_err != cudaSuccess) return;
+      cudaError_t e = cudaFuncGetAttributes(&fa, kernel);
+      if (e == cudaSuccess && fa.numRegs != kLaunchRegs) e = cudaErrorInvalidKernelImage;
+      if (e == cudaSuccess) e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+      if (e != cudaSuccess) return e;
     }
+    return cudaSuccess;
   });
   if (attr_err != cudaSuccess) return attr_err;
 

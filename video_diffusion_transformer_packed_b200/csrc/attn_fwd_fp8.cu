@@ -489,16 +489,15 @@ cudaError_t launch_attn_fp8(const void* qk8, const void* v8t, void* out, int64_t
                             float scale_v, cudaStream_t stream) {
   auto encode = encode_fn();
   if (!encode) return cudaErrorNotSupported;
-  static std::once_flag attr_once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(attr_once, [] {
+  static PerDeviceOnce setup;
+  const cudaError_t attr_err = setup.run([](int) {
     cudaFuncAttributes fa;
-    attr_err = cudaFuncGetAttributes(&fa, attn_fwd_fp8_kernel);
-    if (attr_err == cudaSuccess && fa.numRegs != kLaunchRegs) attr_err = cudaErrorInvalidKernelImage;
-    if (attr_err == cudaSuccess) {
-      attr_err = cudaFuncSetAttribute(attn_fwd_fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      kSmemBytes);
+    cudaError_t e = cudaFuncGetAttributes(&fa, attn_fwd_fp8_kernel);
+    if (e == cudaSuccess && fa.numRegs != kLaunchRegs) e = cudaErrorInvalidKernelImage;
+    if (e == cudaSuccess) {
+      e = cudaFuncSetAttribute(attn_fwd_fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     }
+    return e;
   });
   if (attr_err != cudaSuccess) return attr_err;
 

@@ -309,16 +309,18 @@ cudaError_t launch_gemm_bf16(const void* x, const void* w, void* y, int64_t M, i
                              double* stats, int64_t stat_cols, cudaStream_t stream) {
   auto encode = gemm_encode_fn();
   if (!encode) return cudaErrorNotSupported;
-  static std::once_flag attr_once;
-  static cudaError_t attr_err = cudaSuccess;
-  static int sms = 148;
-  std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(gemm_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    int dev = 0;
-    if (attr_err == cudaSuccess) attr_err = cudaGetDevice(&dev);
-    if (attr_err == cudaSuccess) attr_err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  });
+  static PerDeviceOnce setup;
+  static int sms_of[kMaxDevices];
+  int dev = 0;
+  const cudaError_t attr_err = setup.run(
+      [](int d) {
+        cudaError_t e = cudaFuncSetAttribute(gemm_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms_of[d], cudaDevAttrMultiProcessorCount, d);
+        return e;
+      },
+      &dev);
   if (attr_err != cudaSuccess) return attr_err;
+  const int sms = sms_of[dev];
   alignas(64) CUtensorMap map_x, map_w;
   cuuint32_t box[2] = {kKStep, 128};
   cuuint32_t estr[2] = {1, 1};

@@ -38,7 +38,6 @@ struct DeviceQueues {
   std::vector<cudaEvent_t> events;
 };
 
-constexpr int kMaxDevices = 64;
 DeviceQueues g_queues[kMaxDevices];
 
 cudaError_t ensure_queues(DeviceQueues& q, size_t n_events) {

@@ -43,6 +43,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <mutex>
 
 #include "sm100.cuh"
 #include "wan_kernels.h"
@@ -487,22 +488,42 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const __grid_
 
 template <int VPT, bool kStats>
 cudaError_t launch_vpt(const NormRopeParams& p, uint32_t smem_bytes, cudaStream_t stream) {
-  static int blocks_per_sm = -1;  // per instantiation; the smem size is fixed per instantiation
-  static uint32_t configured_smem = 0;
-  if (configured_smem != smem_bytes) {
-    cudaError_t e = cudaFuncSetAttribute(qk_norm_rope_kernel<VPT, kStats>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem_bytes));
-    if (e != cudaSuccess) return e;
-    int n = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, qk_norm_rope_kernel<VPT, kStats>, kThreads, smem_bytes);
-    if (e != cudaSuccess) return e;
-    blocks_per_sm = n > 0 ? n : 1;
-    configured_smem = smem_bytes;
-  }
-  int dev = 0, sms = 0;
+  // Per device: the dynamic shared-memory limit set so far and the
+  // occupancy at the last size (the size depends on the hidden width).
+  struct DeviceState {
+    uint32_t attr_smem = 0, occ_smem = 0;
+    int blocks_per_sm = 1, sms = 0;
+  };
+  static std::mutex mu;
+  static DeviceState state[kMaxDevices];
+  int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
-  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  int blocks_per_sm = 1, sms = 0;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    DeviceState& st = state[dev];
+    if (st.sms == 0) {
+      e = cudaDeviceGetAttribute(&st.sms, cudaDevAttrMultiProcessorCount, dev);
+      if (e != cudaSuccess) return e;
+    }
+    if (st.attr_smem < smem_bytes) {
+      e = cudaFuncSetAttribute(qk_norm_rope_kernel<VPT, kStats>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem_bytes));
+      if (e != cudaSuccess) return e;
+      st.attr_smem = smem_bytes;
+    }
+    if (st.occ_smem != smem_bytes) {
+      int n = 0;
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, qk_norm_rope_kernel<VPT, kStats>, kThreads, smem_bytes);
+      if (e != cudaSuccess) return e;
+      st.blocks_per_sm = n > 0 ? n : 1;
+      st.occ_smem = smem_bytes;
+    }
+    blocks_per_sm = st.blocks_per_sm;
+    sms = st.sms;
+  }
   const int64_t want = static_cast<int64_t>(sms) * blocks_per_sm;
   const int64_t blocks = p.tokens < want ? p.tokens : want;
   qk_norm_rope_kernel<VPT, kStats><<<static_cast<unsigned>(blocks), kThreads, smem_bytes, stream>>>(p);

@@ -4,8 +4,30 @@
 
 #include <cstdint>
 #include <cuda_runtime.h>
+#include <mutex>
 
 namespace wan {
+
+constexpr int kMaxDevices = 64;
+
+// One-time setup of a launcher per device (function attributes such as the
+// dynamic shared-memory limit are set per device): run() calls init(dev)
+// once for the calling thread's current device, thread-safe, and returns
+// that call's result every time after.
+struct PerDeviceOnce {
+  std::once_flag flag[kMaxDevices];
+  cudaError_t result[kMaxDevices] = {};
+  template <class F>
+  cudaError_t run(F&& init, int* dev_out = nullptr) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::call_once(flag[dev], [&] { result[dev] = init(dev); });
+    if (dev_out != nullptr) *dev_out = dev;
+    return result[dev];
+  }
+};
 
 // Q/K RMSNorm + bf16 round + 3D RoPE, in place on the packed buffer.
 // Arguments are assumed validated by the ABI layer.

@@ -5,6 +5,7 @@ a closed form, an invariant of the mathematics, or brute force.
 Steps pinned (see oracle/wan_oracle.c):
   bf16 rounding          -> torch's float32->bf16 conversion (RNE) on float32 inputs
   RMSNorm over full D    -> torch.nn.functional.rms_norm in fp64; constant-row closed form;
+                            unit-gamma mean square; scale invariance up to eps;
                             per-head-magnitude input separates full-width from per-head
   gamma indexing         -> per-head distinct gammas scale exactly their head
   rounding point         -> token 0 (zero angle) equals round(norm) bit for bit
@@ -69,6 +70,35 @@ def test_rmsnorm_constant_row_closed_form():
     assert np.allclose(got, 0.5 / math.sqrt(0.25 + 1e-6), rtol=1e-15, atol=0)
     # and eps matters at this precision (guards a dropped eps)
     assert abs(got[0, 0] - 1.0) > 1e-7
+
+
+def test_rmsnorm_unit_gamma_gives_unit_mean_square():
+    """With gamma = 1, mean(y^2) = ms / (ms + eps) exactly in real arithmetic:
+    1 up to eps / ms (a dropped mean, a sum instead of the mean, or a missing
+    square root all break it)."""
+    heads = 4
+    x = wi.packed_qkv(1, 9, heads, seed=21)[0, :, : heads * HD]
+    g = torch.ones(heads * HD).to(torch.bfloat16)
+    y = oracle.rmsnorm(x, g, EPS)
+    ms = (x.double().numpy() ** 2).mean(axis=1)
+    np.testing.assert_allclose((y ** 2).mean(axis=1), ms / (ms + EPS), rtol=1e-13, atol=0)
+    assert np.all(np.abs((y ** 2).mean(axis=1) - 1.0) < 2e-6)
+
+
+def test_rmsnorm_scale_invariance_up_to_eps():
+    """y(c x) = x / sqrt(ms + eps / c^2): scaling the row by c = 4 (exact in
+    bf16) leaves y unchanged up to the eps term, and the change has the sign
+    and size eps predicts."""
+    heads = 2
+    x = wi.packed_qkv(1, 5, heads, seed=22)[0, :, : heads * HD]
+    gq, _ = wi.gammas(heads, 6, 7)
+    y1 = oracle.rmsnorm(x, gq, EPS)
+    y4 = oracle.rmsnorm((x.double() * 4).to(torch.bfloat16), gq, EPS)
+    ms = (x.double().numpy() ** 2).mean(axis=1, keepdims=True)
+    # |y4| / |y1| = sqrt((ms + eps) / (ms + eps / 16)) > 1
+    ratio = np.sqrt((ms + EPS) / (ms + EPS / 16))
+    np.testing.assert_allclose(y4, y1 * ratio, rtol=1e-13, atol=0)
+    assert np.all(ratio > 1.0) and np.all(ratio - 1.0 < 1e-6)
 
 
 def test_rmsnorm_is_full_width_not_per_head():

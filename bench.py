@@ -516,6 +516,9 @@ def run_ours(args):
                    "step": "wan_dit_attn: qk_norm_rope in place, then attention (PDL-chained)"},
         "attn_tflops": attn_tflops, "attn_frac_of_peak": attn_tflops / tensor_peak,
         "norm_rope_gbs": norm_gbs, "norm_rope_frac_of_hbm": norm_gbs / peaks["hbm_gbs"],
+        # the fused call (one step, PDL-chained) against its two kernels timed
+        # as separate calls on the same stream
+        "fused": {"step_ms": ms_step, "norm_ms": t_norm, "attn_ms": t_attn, "parts_sum_ms": t_norm + t_attn},
         "roofline": roofline, "roofline_norm_rope": norm_roofline,
         "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks, "skip_softmax": skip, "fp8": fp8,
         "qkv_projection": proj,

@@ -77,11 +77,13 @@ typedef enum {
                                      is not memory of the current device */
 } wan_status;
 
-/* wan_dit_attn_host flag: the copies into qkv_dev start without waiting for
- * earlier work on `stream`. The caller guarantees that no earlier work still
- * uses qkv_dev or out_dev (e.g. it alternates two sets between consecutive
- * calls), so that one call's input transfer overlaps the previous call's
- * kernels. */
+/* wan_dit_attn_host flag: the call does not wait for earlier work on
+ * `stream`. Its copies into qkv_dev still wait for the kernels of earlier
+ * wan_dit_attn_host calls that read the same qkv_dev, and its kernels wait for
+ * those calls' copies out of the same out_dev; nothing else orders them. The
+ * caller guarantees that no other earlier work still uses qkv_dev or out_dev.
+ * A caller that alternates two buffer sets between consecutive calls gets one
+ * call's input transfer overlapped with the previous call's kernels. */
 #define WAN_HOST_OVERLAP_INPUT 1
 
 /* Default head-chunk size of wan_dit_attn_host's pipeline. */
@@ -251,14 +253,15 @@ WAN_API int32_t wan_dit_attn(void* qkv, void* out, int64_t batch, int32_t F, int
 
 /*
  * (1) then (2) for packed QKV and output that live in HOST memory: the call
- * a user with host-resident activations makes. Copies and kernels overlap
- * chunk by chunk, because PCIe, not the kernels, bounds this step:
- *  - per batch element, the Q|K channels of every token are copied first
- *    (the RMS of (1) runs over all heads of a token), then (1) runs on that
- *    batch element;
- *  - V follows in chunks of heads_per_chunk heads, and (2) for a head chunk
- *    starts as soon as its V chunk has arrived;
- *  - each head chunk of `out` is copied back while later chunks compute.
+ * a user with host-resident activations makes. The PCIe transfers and the
+ * kernels bound this step about equally, so they overlap:
+ *  - each batch element's packed rows are copied in one contiguous copy (the
+ *    fastest pattern over PCIe), and (1) runs on the element once they have
+ *    arrived, while the next element's copy proceeds;
+ *  - (2) follows in chunks of heads_per_chunk heads, and each head chunk of
+ *    `out` is copied back while later chunks compute;
+ *  - with WAN_HOST_OVERLAP_INPUT, consecutive calls on alternating buffer
+ *    sets also overlap one call's copies with the previous call's kernels.
  * qkv_host  page-locked host memory (cudaHostAlloc / cudaHostRegister), bf16
  *           [batch][F*H*W][3*heads*128]; only read.
  * out_host  page-locked host memory, bf16 [batch][F*H*W][heads*128]; written.
@@ -271,13 +274,13 @@ WAN_API int32_t wan_dit_attn(void* qkv, void* out, int64_t batch, int32_t F, int
  *           heads); batch * ceil(heads/heads_per_chunk) <= WAN_HOST_MAX_PIECES.
  * flags     0 or WAN_HOST_OVERLAP_INPUT.
  * Other arguments as for wan_dit_attn. Device pointers 16-byte aligned.
- * Execution: asynchronous and ordered on `stream`: the copies into qkv_dev
- * start after the work enqueued on `stream` before this call (unless
- * WAN_HOST_OVERLAP_INPUT), and work
+ * Execution: asynchronous. The call's copies and kernels start after the work
+ * enqueued on `stream` before it (unless WAN_HOST_OVERLAP_INPUT), and work
  * enqueued on `stream` after it runs once out_host is written (synchronise
- * `stream` before reading out_host on the host). The library keeps two
- * internal streams per device for the copies; concurrent calls on one device
- * are serialised while they are enqueued.
+ * `stream` before reading out_host on the host). The library runs the copies
+ * in and out and the kernels on three internal streams per device. Calls on
+ * one device are serialised while they are enqueued, and their kernels run in
+ * that order.
  * Errors: argument errors return before anything is enqueued, as for the other
  * calls; WAN_ERR_MEMORY_KIND when a host buffer is not page-locked or a device
  * buffer is not memory of the current device; WAN_ERR_LAUNCH when the runtime

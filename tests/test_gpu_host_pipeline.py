@@ -135,3 +135,30 @@ def test_overlapped_calls_with_alternating_buffers():
     s.synchronize()
     for o, r in zip(outs, refs):
         assert torch.equal(o.view(torch.int16), r.view(torch.int16))
+
+
+@pytest.mark.parametrize("n_sets", [2, 1])
+def test_overlapped_calls_when_kernels_outlast_the_transfer(n_sets):
+    """One head at S = 75600: each call's attention takes about twice its input
+    transfer, so the copy stream runs ahead of the kernels. Eight overlapped
+    calls on two alternating buffer sets (or one set reused by every call):
+    a call's copies into a set must wait for the kernels of the call that used
+    it before, and every output must equal the device path's."""
+    w = wi.Workload("case", 1, (21, 45, 80), 1)
+    gq_h, gk_h = wi.gammas(w.heads)
+    gq, gk = gq_h.cuda(), gk_h.cuda()
+    s = torch.cuda.Stream()
+    sets = [(torch.empty((w.batch, w.seq_len, 3 * w.dim), dtype=torch.bfloat16, device="cuda"),
+             torch.empty((w.batch, w.seq_len, w.dim), dtype=torch.bfloat16, device="cuda"))
+            for _ in range(n_sets)]
+    inputs = [_pinned(wi.packed_qkv(w.batch, w.seq_len, w.heads, seed=40 + k)) for k in range(8)]
+    refs = [_device_reference(x.clone(), w, gq, gk)[1].cpu() for x in inputs]
+    outs = []
+    for k, x in enumerate(inputs):
+        qd, od = sets[k % n_sets]
+        outs.append(wan.dit_attn_host(x, w.grid, w.heads, gq, gk, qkv_dev=qd, out_dev=od,
+                                      overlap_input=True, stream=s))
+    s.synchronize()
+    assert wan.device_error() == 0
+    for o, r in zip(outs, refs):
+        assert torch.equal(o.view(torch.int16), r.view(torch.int16))

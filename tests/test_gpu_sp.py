@@ -61,3 +61,24 @@ def test_query_row_ranges_at_ragged_offsets():
         got = wan.self_attention_rows(d, w.heads, r0, n)
         torch.cuda.synchronize()
         assert torch.equal(got.view(torch.int16), ref[:, r0:r0 + n].view(torch.int16))
+
+
+def test_shards_starting_mid_row_with_many_batch_boundaries():
+    """Shards of 525 tokens (3.5 rows of 150) over a batch of 40: every CTA's
+    token range crosses batch boundaries, where the shard's grid positions
+    restart at s0, and long column runs step the rotations one by one; the
+    shards must reproduce the full-buffer norm+RoPE bit for bit."""
+    grid, heads, batch, world = (2, 7, 150), 1, 40, 4
+    S = grid[0] * grid[1] * grid[2]
+    qkv = wi.packed_qkv(batch, S, heads, seed=31)
+    gq, gk = wi.gammas(heads, 32, 33)
+    gq, gk = gq.cuda(), gk.cuda()
+    ref = qkv.cuda()
+    wan.qk_norm_rope(ref, grid, heads, gq, gk)
+    s_local = S // world
+    shards = [qkv[:, r * s_local:(r + 1) * s_local].contiguous().cuda() for r in range(world)]
+    for r, sh in enumerate(shards):
+        wan.qk_norm_rope_shard(sh, grid, heads, r * s_local, gq, gk)
+    torch.cuda.synchronize()
+    assert wan.device_error() == 0
+    assert torch.equal(torch.cat(shards, dim=1).view(torch.int16), ref.view(torch.int16))

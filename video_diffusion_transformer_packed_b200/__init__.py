@@ -362,8 +362,11 @@ def dit_attn_host(qkv_host, grid: Sequence[int], heads: int, gamma_q, gamma_k, o
     overlapped chunk by chunk inside the library. qkv_dev / out_dev are the
     device buffers it runs through (allocated on the current device when not
     given); qkv_host is only read. Asynchronous on `stream`: synchronise it
-    before reading out_host. overlap_input: the input transfer does not wait
-    for earlier work on `stream` (the caller alternates device buffer sets)."""
+    before reading out_host. overlap_input: the call does not wait for earlier
+    work on `stream`; it still waits for earlier calls of this function that
+    use the same device buffers (the caller guarantees nothing else does), so
+    alternating two buffer sets overlaps one call's input transfer with the
+    previous call's kernels."""
     import torch
     F, H, W = grid
     _check_packed(qkv_host, heads, grid)

@@ -85,7 +85,7 @@ struct HostStep {
   const void* gamma_q;
   const void* gamma_k;
   float eps, theta, scale;
-  bool overlap_input;  // copies in do not wait for earlier work on the stream
+  bool overlap_input;  // no wait for earlier work on the stream (buffer fences only)
 };
 cudaError_t enqueue_dit_attn_host(const HostStep& step, cudaStream_t stream);
 

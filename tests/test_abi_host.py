@@ -189,3 +189,43 @@ def test_sequence_shard_entry_points_validate(lib):
     assert lib.wan_self_attention_rows(FAKE, 2**40, 1, 8, 1, 128, 6, 3, 0.0, None) == 3
     assert lib.wan_self_attention_rows(FAKE, 2**40, 1, 8, 1, 128, 0, 0, 0.0, None) == 3
     assert lib.wan_self_attention_rows(FAKE, FAKE + 64, 1, 8, 1, 128, 0, 4, 0.0, None) == 9
+
+
+C_CALLER = r"""
+#include <stdio.h>
+#include "wan_attn.h"
+
+int main(void) {
+  int32_t s;
+  printf("abi %d\n", (int)wan_abi_version());
+  for (s = 0; s <= 10; ++s) printf("status %d %s\n", (int)s, wan_status_string(s));
+  /* argument errors are reported before any CUDA call */
+  printf("null %d\n", (int)wan_qk_norm_rope(NULL, 1, 1, 1, 1, 1, 128, NULL, NULL, 1e-6f, 1e4f, NULL));
+  printf("head_dim %d\n", (int)wan_self_attention((const void*)16, (void*)4096, 1, 1, 1, 64, 0.f, NULL));
+  return 0;
+}
+"""
+
+
+def test_header_compiles_as_c_and_links(lib, tmp_path):
+    """A plain C99 caller: the header compiles with warnings as errors, the
+    program links against the library, and the calls that need no GPU answer
+    (ABI version, status text, argument validation)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "caller.c"
+    src.write_text(C_CALLER)
+    exe = tmp_path / "caller"
+    libdir = os.path.dirname(wan.library_path())
+    subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-o", str(exe), "-L", libdir, "-l:" + os.path.basename(wan.library_path()),
+                    "-Wl,-rpath," + libdir], check=True, capture_output=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.splitlines()
+    assert out[0] == f"abi {lib.wan_abi_version()}"
+    texts = [line.split(" ", 2)[2] for line in out[1:12]]
+    assert all(texts) and len(set(texts)) == 11
+    assert out[12] == "null 1"          # WAN_ERR_NULL
+    assert out[13] == "head_dim 4"      # WAN_ERR_HEAD_DIM

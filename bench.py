@@ -232,7 +232,9 @@ def run_reference(args):
         "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1000.0 * statistics.mean(times), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {**w.describe(), "sample": desc},
+        # the GPU arm's workload keys, plus what this arm actually timed
+        "config": {**w.describe(), "parallelism": f"replicas{args.gpus}" if args.gpus > 1 else "single",
+                   "step": "norm+RoPE and attention of the step, fp64 oracle on a bounded sample", "sample": desc},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }

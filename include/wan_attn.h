@@ -73,8 +73,11 @@ typedef enum {
   WAN_ERR_LAUNCH = 7,             /* the CUDA runtime rejected a launch */
   WAN_ERR_DEVICE_TIMEOUT = 8,     /* a kernel's bounded wait gave up (see wan_device_error) */
   WAN_ERR_ALIAS = 9,              /* out overlaps qkv */
-  WAN_ERR_MEMORY_KIND = 10        /* a host buffer is not page-locked, or a device buffer
+  WAN_ERR_MEMORY_KIND = 10,       /* a host buffer is not page-locked, or a device buffer
                                      is not memory of the current device */
+  WAN_ERR_KERNEL_IMAGE = 11       /* a compiled attention kernel's register count differs from
+                                     the one its per-warpgroup register split was written for
+                                     (a toolkit other than the one the library targets) */
 } wan_status;
 
 /* wan_dit_attn_host flag: the call does not wait for earlier work on
@@ -146,7 +149,9 @@ WAN_API int32_t wan_self_attention(const void* qkv, void* out, int64_t batch, in
  * weighted sums; when all four groups of a query tile skip, the P V product
  * is not run. Tile 0 is never skipped; a group holding rows past seq_len
  * never skips. threshold == 0 runs the dense kernel (bit-identical to
- * wan_self_attention); threshold must be finite and >= 0.
+ * wan_self_attention); 0 <= threshold <= 1 (a weight is compared with the
+ * row's largest one, so a threshold above 1 would also drop tiles that hold
+ * the row's maximum), else WAN_ERR_PARAM.
  * Other arguments as for wan_self_attention. Counters of what was skipped:
  * wan_skip_stats.
  */
@@ -233,11 +238,53 @@ WAN_API int32_t wan_self_attention_rows(const void* qkv, void* out, int64_t batc
                                         int32_t head_dim, int64_t q_row0, int64_t q_rows, float scale, void* stream);
 
 /*
- * Synchronises `stream`, then reads and clears the Skip-Softmax counters
- * accumulated by wan_self_attention_sparse launches since the last read:
- * *group_tiles = (32-row group, key tile) pairs skipped, *products = 128-row
- * P V products skipped. Either pointer may be NULL. Returns WAN_ERR_LAUNCH
- * when the synchronisation reports a CUDA error.
+ * Context parallelism in ring form (the fourth NEXT item; AWS Neuron page,
+ * "Context parallelism" and "NKI kernels": each rank keeps its S/N shard of Q
+ * and of K/V, the K/V chunks travel around the ring, and each round's
+ * attention, overlapped with the next exchange, is folded into the rank's
+ * running result; the page's kernel for this is ring_attention_const_max_fwd).
+ * A round's result is the online-softmax state of one key range, and states
+ * over disjoint ranges combine exactly:
+ *
+ * wan_self_attention_partial: (2) for query rows [q_row0, q_row0 + q_rows) of
+ *   q_qkv (packed, [batch][q_seq_len][3*heads*128]) against the keys
+ *   [k_row0, k_row0 + k_rows) of kv ([batch][kv_rows][kv_pitch] bf16 whose
+ *   last 2*heads*128 columns hold K then V: kv_pitch = 3*heads*128 for a packed
+ *   QKV buffer, 2*heads*128 for a K|V chunk). Instead of the normalised bf16
+ *   output it writes the softmax state of that key range, per (row, head):
+ *     o  [batch][q_rows][heads][128] fp32: O = sum_j 2^(a_j - m) v_j
+ *     ml [batch][q_rows][heads][2]   fp32: (m, l = sum_j 2^(a_j - m))
+ *   with a_j = scale * log2(e) * q . k_j (scale <= 0: 1/sqrt(128)) and m a
+ *   reference maximum chosen by the kernel (at most 8 below the largest a_j).
+ *   O uses the probabilities rounded to bf16, as (2) does, and so does l.
+ *   All pointers 16-byte aligned; o and ml overlap neither input nor each
+ *   other. The full row's output is merge(all ranges) finalised below.
+ * wan_attention_merge: for n_units (row, head) units in the layouts above
+ *   (n_units = batch * rows * heads): when o_part is not NULL,
+ *   (o_acc, ml_acc) := the merge of itself and (o_part, ml_part):
+ *     m = max(m_acc, m_part), O = 2^(m_acc - m) O_acc + 2^(m_part - m) O_part,
+ *     l likewise;
+ *   then, when out is not NULL, out = bf16(O_acc / l_acc), 128 bf16 per unit
+ *   (for units ordered [batch][rows][heads]: wan_self_attention's layout).
+ *   o_part and ml_part are both given or both NULL; o_part and out are not
+ *   both NULL. No buffer overlaps another. head_dim == 128.
+ */
+WAN_API int32_t wan_self_attention_partial(const void* q_qkv, int64_t q_seq_len, int64_t q_row0, int64_t q_rows,
+                                           const void* kv, int64_t kv_rows, int64_t kv_pitch, int64_t k_row0,
+                                           int64_t k_rows, float* o, float* ml, int64_t batch, int32_t heads,
+                                           int32_t head_dim, float scale, void* stream);
+WAN_API int32_t wan_attention_merge(float* o_acc, float* ml_acc, const float* o_part, const float* ml_part,
+                                    void* out, int64_t n_units, int32_t head_dim, void* stream);
+
+/*
+ * Reads and clears the Skip-Softmax counters: *group_tiles = (32-row group,
+ * key tile) pairs skipped, *products = 128-row P V products skipped. The
+ * counters are one pair per device, shared by every wan_self_attention_sparse
+ * launch on it (any stream, any host thread): a read returns what all of them
+ * counted since the previous read. The read and the clear are one atomic
+ * exchange, done on `stream` after the work enqueued on it before this call;
+ * the call then synchronises `stream`. Either pointer may be NULL. Returns
+ * WAN_ERR_LAUNCH when the stream reports a CUDA error.
  */
 WAN_API int32_t wan_skip_stats(void* stream, int64_t* group_tiles, int64_t* products);
 
@@ -294,13 +341,18 @@ WAN_API int32_t wan_dit_attn_host(const void* qkv_host, void* out_host, void* qk
                                   int32_t flags, void* stream);
 
 /*
- * Synchronises `stream`, then reads and clears the device-side error words
- * that the kernels set when one of their bounded waits gives up. *code
- * receives 0 when no wait gave up, otherwise a nonzero value: the bf16
- * attention's site code in bits 0-7, norm+RoPE's in bits 8-15, the FP8
- * attention's in bits 16-23, the projection GEMM's in bits 24-30.
+ * Reads and clears the device-side error words that the kernels set when one
+ * of their bounded waits gives up. *code receives 0 when no wait gave up,
+ * otherwise a nonzero value: the bf16 attention's site code in bits 0-7,
+ * norm+RoPE's in bits 8-15, the FP8 attention's in bits 16-23, the projection
+ * GEMM's in bits 24-30. The words are one set per device, shared by every
+ * launch on it (any stream, any host thread): a read reports and clears what
+ * any of them recorded since the previous read, so a caller that needs to
+ * know which call failed keeps other work off the device meanwhile. The read
+ * and the clear are one atomic exchange per word, done on `stream` after the
+ * work enqueued on it before this call; the call then synchronises `stream`.
  * Returns WAN_ERR_DEVICE_TIMEOUT when *code != 0, WAN_ERR_NULL when code is
- * NULL, WAN_ERR_LAUNCH when the synchronisation reports a CUDA error.
+ * NULL, WAN_ERR_LAUNCH when the stream reports a CUDA error.
  */
 WAN_API int32_t wan_device_error(void* stream, int32_t* code);
 

@@ -54,6 +54,7 @@ def _load():
             lib.wan_oracle_qk_norm_rope_tokens.argtypes = [P, I64, I32, I32, I32, I32, P, P, D, D,
                                                            P, I64, P]
             lib.wan_oracle_attention_rows.argtypes = [P, I64, I64, I32, D, P, I64, P]
+            lib.wan_oracle_attention_partial_rows.argtypes = [P, I64, P, I64, I64, I64, I64, I32, D, P, I64, P, P]
             lib.wan_oracle_attention_skip_groups.argtypes = [P, I64, I64, I32, D, D, P, I64, P, P, P]
             lib.wan_oracle_e4m3_encode.argtypes = [D]
             lib.wan_oracle_e4m3_encode.restype = ctypes.c_uint8
@@ -152,6 +153,43 @@ def attention_rows(qkv: torch.Tensor, heads: int, rows, scale: float) -> np.ndar
     return out
 
 
+def attention_partial_rows(q_qkv: torch.Tensor, heads: int, kv: torch.Tensor, k_row0: int, k_rows: int, rows,
+                           scale: float):
+    """Step 4 over the keys [k_row0, k_row0 + k_rows) of kv [B, Skv, pitch]
+    (K then V in its last 2*heads*128 columns) for listed (b, h, i) rows of the
+    packed q_qkv: the softmax state (o fp64 [n, 128], ml fp64 [n, 2] = (m, l)),
+    o = sum_j exp(a_j - m) v_j, l = sum_j exp(a_j - m), m = max_j a_j."""
+    B, Sq, D3 = q_qkv.shape
+    assert D3 == 3 * heads * HEAD_DIM and kv.shape[0] == B and kv.shape[2] >= 2 * heads * HEAD_DIM
+    assert 0 <= k_row0 and k_rows >= 1 and k_row0 + k_rows <= kv.shape[1]
+    r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 3))
+    assert (r[:, 0] < B).all() and (r[:, 1] < heads).all() and (r[:, 2] < Sq).all() and (r >= 0).all()
+    o = np.empty((r.shape[0], HEAD_DIM), dtype=np.float64)
+    ml = np.empty((r.shape[0], 2), dtype=np.float64)
+    qb, kb = _bits(q_qkv), _bits(kv)
+    _load().wan_oracle_attention_partial_rows(_ptr(qb), Sq, _ptr(kb), kv.shape[1], kv.shape[2], int(k_row0),
+                                              int(k_rows), heads, float(scale), _ptr(r), r.shape[0], _ptr(o),
+                                              _ptr(ml))
+    return o, ml
+
+
+def merge_partial(a, b):
+    """Two softmax states over disjoint key ranges -> the state over their
+    union (fp64): m = max(m_a, m_b), each side scaled by exp(its m - m)."""
+    (oa, mla), (ob, mlb) = a, b
+    m = np.maximum(mla[..., 0], mlb[..., 0])
+    wa, wb = np.exp(mla[..., 0] - m), np.exp(mlb[..., 0] - m)
+    o = oa * wa[..., None] + ob * wb[..., None]
+    ml = np.stack([m, mla[..., 1] * wa + mlb[..., 1] * wb], axis=-1)
+    return o, ml
+
+
+def finalize_partial(state) -> np.ndarray:
+    """The attention output of a softmax state: o / l."""
+    o, ml = state
+    return o / ml[..., 1:2]
+
+
 def attention_skip_groups(qkv: torch.Tensor, heads: int, groups, scale: float, threshold: float):
     """Step 4 with Skip-Softmax (threshold mode) for listed (b, h, g) groups of
     32 query rows: (out fp64 [n, 32, 128] (rows past S: NaN), skipped bool
@@ -222,6 +260,18 @@ def linear_rows(x: torch.Tensor, w: torch.Tensor, rows) -> np.ndarray:
     Wan2.2 Dataflow": the fused QKV projection output is the packed buffer)."""
     xr = x.reshape(-1, x.shape[-1])[torch.as_tensor(np.asarray(rows, dtype=np.int64))].double().numpy()
     return xr @ w.double().numpy().T
+
+
+def linear_bf16(x: torch.Tensor, w: torch.Tensor, chunk: int = 4096) -> torch.Tensor:
+    """The projection Y = X W^T for every row of X [M, K], each output rounded
+    once to bf16 (RNE): the packed buffer as the projection stores it.
+    Evaluated `chunk` rows at a time with linear_rows."""
+    M = x.reshape(-1, x.shape[-1]).shape[0]
+    out = torch.empty((M, w.shape[0]), dtype=torch.bfloat16)
+    for r0 in range(0, M, chunk):
+        r1 = min(r0 + chunk, M)
+        out[r0:r1] = to_bf16(linear_rows(x, w, np.arange(r0, r1)))
+    return out
 
 
 def attention_full(qkv: torch.Tensor, heads: int, scale: float) -> np.ndarray:

@@ -229,6 +229,58 @@ void wan_oracle_attention_rows(const uint16_t* qkv, int64_t batch, int64_t S, in
   }
 }
 
+/* Step 4 for one key range, as one round of ring context parallelism
+ * (AWS Neuron "Optimizing High-Quality Offline Video Generation", "Context
+ * parallelism": each rank's queries meet the K/V chunks one at a time, and
+ * the rounds' results are combined). For each listed query row (b, h, i) of
+ * q_qkv (packed [B, Sq, 3, heads, 128]) and the keys [k_row0, k_row0 + k_rows)
+ * of kv ([B, kv_rows, kv_pitch], K then V in the last 2*heads*128 columns):
+ *     a_j = scale * q_i . k_j,  m = max_j a_j,
+ *     l = sum_j exp(a_j - m),    o = sum_j exp(a_j - m) v_j        (fp64)
+ * o: n x 128, ml: n x 2 (m, l), natural-log units. The softmax of the range
+ * is o / l; two ranges' states merge as in oracle.merge_partial. */
+void wan_oracle_attention_partial_rows(const uint16_t* q_qkv, int64_t Sq, const uint16_t* kv, int64_t kv_rows,
+                                       int64_t kv_pitch, int64_t k_row0, int64_t k_rows, int32_t heads,
+                                       double scale, const int64_t* rows, int64_t n, double* o, double* ml) {
+  const int64_t D = (int64_t)heads * HEAD_DIM, D3 = 3 * D;
+  const int64_t k_col = kv_pitch - 2 * D, v_col = kv_pitch - D;
+#pragma omp parallel
+  {
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t r = 0; r < n; ++r) {
+      int64_t b = rows[3 * r], h = rows[3 * r + 1], i = rows[3 * r + 2];
+      const uint16_t* qrow = q_qkv + (b * Sq + i) * D3 + h * HEAD_DIM;
+      const uint16_t* kvb = kv + b * kv_rows * kv_pitch;
+      double q[HEAD_DIM];
+      for (int d = 0; d < HEAD_DIM; ++d) q[d] = bf16_to_f64(qrow[d]);
+      /* pass 1: the largest logit of the range */
+      double m = -INFINITY;
+      for (int64_t j = k_row0; j < k_row0 + k_rows; ++j) {
+        const uint16_t* k = kvb + j * kv_pitch + k_col + h * HEAD_DIM;
+        double dot = 0.0;
+        for (int d = 0; d < HEAD_DIM; ++d) dot += q[d] * bf16_to_f64(k[d]);
+        if (dot * scale > m) m = dot * scale;
+      }
+      /* pass 2: exponentials, their sum and the weighted sum of V */
+      double acc[HEAD_DIM];
+      for (int d = 0; d < HEAD_DIM; ++d) acc[d] = 0.0;
+      double sum = 0.0;
+      for (int64_t j = k_row0; j < k_row0 + k_rows; ++j) {
+        const uint16_t* k = kvb + j * kv_pitch + k_col + h * HEAD_DIM;
+        const uint16_t* v = kvb + j * kv_pitch + v_col + h * HEAD_DIM;
+        double dot = 0.0;
+        for (int d = 0; d < HEAD_DIM; ++d) dot += q[d] * bf16_to_f64(k[d]);
+        double w = exp(dot * scale - m);
+        sum += w;
+        for (int d = 0; d < HEAD_DIM; ++d) acc[d] += w * bf16_to_f64(v[d]);
+      }
+      for (int d = 0; d < HEAD_DIM; ++d) o[r * HEAD_DIM + d] = acc[d];
+      ml[2 * r] = m;
+      ml[2 * r + 1] = sum;
+    }
+  }
+}
+
 /* Step 4 with Skip-Softmax in threshold mode (vLLM-Omni "Wan2.2 Text-to-Video"
  * recipe, "Accelerating with TRTLLM_ATTN + Skip-Softmax": a direct skip
  * threshold, no calibration). The pages name the threshold but not the rule;

@@ -39,8 +39,8 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings(lib):
-    assert lib.wan_abi_version() == 8
-    for code in range(11):
+    assert lib.wan_abi_version() == 9
+    for code in range(12):
         assert lib.wan_status_string(code)
     assert lib.wan_status_string(99) == b"unknown status"
 
@@ -139,6 +139,9 @@ def test_sparse_attention_validates_threshold(lib):
     # (qkv, out, batch, seq_len, heads, head_dim, scale, threshold)
     assert lib.wan_self_attention_sparse(FAKE, FAKE * 16, 1, 8, 1, 128, 0.0, -0.1, None) == 5
     assert lib.wan_self_attention_sparse(FAKE, FAKE * 16, 1, 8, 1, 128, 0.0, float("nan"), None) == 5
+    # a weight is compared with the row's largest one: a threshold above 1 would drop the maximum
+    assert lib.wan_self_attention_sparse(FAKE, FAKE * 16, 1, 8, 1, 128, 0.0, 1.0001, None) == 5
+    assert lib.wan_self_attention_sparse(FAKE, FAKE * 16, 1, 8, 1, 128, 0.0, 2.0, None) == 5
     assert lib.wan_self_attention_sparse(FAKE, FAKE * 16, 1, 8, 1, 127, 0.0, 0.1, None) == 4
     assert lib.wan_self_attention_sparse(FAKE, FAKE + 64, 1, 8, 1, 128, 0.0, 0.1, None) == 9
 
@@ -180,6 +183,41 @@ def test_linear_validates(lib):
         assert lib.wan_linear(FAKE, FAKE, far, 4, 256, 64, None, 0, None) == 6
 
 
+def test_ring_entry_points_validate(lib):
+    far1, far2, far3 = 2**40, 2**41, 2**42
+    # wan_self_attention_partial(q, Sq, q_row0, q_rows, kv, kv_rows, kv_pitch, k_row0, k_rows, o, ml, B, heads, hd, scale)
+    ok = (FAKE, 8, 0, 8, far1, 8, 256, 0, 8, far2, far3, 1, 1, 128, 0.0, None)
+    def call(**kw):
+        a = list(ok)
+        names = ["q", "Sq", "q0", "qn", "kv", "kvr", "pitch", "k0", "kn", "o", "ml", "B", "h", "hd", "sc", "st"]
+        for k, v in kw.items():
+            a[names.index(k)] = v
+        return lib.wan_self_attention_partial(*a)
+    assert call(q=None) == 1 and call(o=None) == 1
+    assert call(ml=far3 + 8) == 2
+    assert call(hd=64) == 4
+    assert call(q0=4, qn=5) == 3              # query rows past Sq
+    assert call(k0=1, kn=8) == 3              # keys past kv_rows
+    assert call(kn=0) == 3
+    assert call(pitch=128) == 3               # narrower than K|V
+    assert call(pitch=260) == 3               # rows not whole 16-byte units
+    assert call(sc=float("inf")) == 5
+    assert call(o=FAKE + 16) == 9             # o overlaps q
+    assert call(ml=far2 + 64) == 9            # ml overlaps o
+    # wan_attention_merge(o_acc, ml_acc, o_part, ml_part, out, n_units, head_dim)
+    assert lib.wan_attention_merge(far1, far2, None, None, None, 4, 128, None) == 1  # nothing to do
+    assert lib.wan_attention_merge(far1, far2, far3, None, None, 4, 128, None) == 1  # o_part without ml_part
+    assert lib.wan_attention_merge(far1, far2, None, None, far3, 4, 64, None) == 4
+    assert lib.wan_attention_merge(far1, far2, None, None, far3, 0, 128, None) == 3
+    assert lib.wan_attention_merge(far1 + 8, far2, None, None, far3, 4, 128, None) == 2
+    assert lib.wan_attention_merge(far1, far1 + 256, None, None, far3, 4, 128, None) == 9  # ml in o
+    assert lib.wan_attention_merge(far1, far2, None, None, far1 + 1024, 4, 128, None) == 9  # out in o
+    import torch
+    if not torch.cuda.is_available():
+        assert call() == 6
+        assert lib.wan_attention_merge(far1, far2, None, None, far3, 4, 128, None) == 6
+
+
 def test_sequence_shard_entry_points_validate(lib):
     # wan_qk_norm_rope_shard(qkv, batch, F, H, W, s0, s_local, heads, head_dim, gq, gk, eps, theta)
     assert lib.wan_qk_norm_rope_shard(FAKE, 1, 2, 2, 2, 4, 5, 1, 128, FAKE, FAKE, 1e-6, 1e4, None) == 3
@@ -198,7 +236,7 @@ C_CALLER = r"""
 int main(void) {
   int32_t s;
   printf("abi %d\n", (int)wan_abi_version());
-  for (s = 0; s <= 10; ++s) printf("status %d %s\n", (int)s, wan_status_string(s));
+  for (s = 0; s <= 11; ++s) printf("status %d %s\n", (int)s, wan_status_string(s));
   /* argument errors are reported before any CUDA call */
   printf("null %d\n", (int)wan_qk_norm_rope(NULL, 1, 1, 1, 1, 1, 128, NULL, NULL, 1e-6f, 1e4f, NULL));
   printf("head_dim %d\n", (int)wan_self_attention((const void*)16, (void*)4096, 1, 1, 1, 64, 0.f, NULL));
@@ -225,7 +263,7 @@ def test_header_compiles_as_c_and_links(lib, tmp_path):
                     "-Wl,-rpath," + libdir], check=True, capture_output=True)
     out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.splitlines()
     assert out[0] == f"abi {lib.wan_abi_version()}"
-    texts = [line.split(" ", 2)[2] for line in out[1:12]]
-    assert all(texts) and len(set(texts)) == 11
-    assert out[12] == "null 1"          # WAN_ERR_NULL
-    assert out[13] == "head_dim 4"      # WAN_ERR_HEAD_DIM
+    texts = [line.split(" ", 2)[2] for line in out[1:13]]
+    assert all(texts) and len(set(texts)) == 12
+    assert out[13] == "null 1"          # WAN_ERR_NULL
+    assert out[14] == "head_dim 4"      # WAN_ERR_HEAD_DIM

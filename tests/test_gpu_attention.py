@@ -50,10 +50,15 @@ def test_tiny_wan_grid_after_oracle_norm_rope():
 
 
 def test_batches_do_not_leak():
-    """Two batches with different content; rows past S in the last tile must
-    read as zeros of the same batch, not the next batch's tokens."""
+    """Two batches with different content and magnitudes (batch 1: queries
+    doubled, so its softmax is sharper, and values halved); rows past S in the
+    last tile must read as zeros of the same batch, not the next batch's tokens."""
     S, heads = 200, 3
-    qkv = torch.cat([wi.packed_qkv(1, S, heads, seed=3), wi.packed_qkv(1, S, heads, seed=33)])
+    D = heads * HD
+    second = wi.packed_qkv(1, S, heads, seed=33).float()
+    second[..., :D] *= 2.0
+    second[..., 2 * D:] *= 0.5
+    qkv = torch.cat([wi.packed_qkv(1, S, heads, seed=3), second.to(torch.bfloat16)])
     got = gpu_attention(qkv, heads)
     ref = oracle.attention_full(qkv, heads, SCALE)
     assert_attention_close(got.view(2, S, heads, HD), ref, "batch")
@@ -68,7 +73,7 @@ def test_peaked_logits_force_rescaling():
     qkv = qkv.to(torch.bfloat16)
     got = gpu_attention(qkv, heads)
     ref = oracle.attention_full(qkv, heads, SCALE)
-    assert_attention_close(got.view(1, S, heads, HD), ref, "peaked", scaled=True)
+    assert_attention_close(got.view(1, S, heads, HD), ref, "peaked")
 
 
 def test_large_scale_spread_logits():
@@ -76,7 +81,7 @@ def test_large_scale_spread_logits():
     qkv = wi.packed_qkv(1, S, heads, seed=5)
     got = gpu_attention(qkv, heads, scale=0.5)
     ref = oracle.attention_full(qkv, heads, 0.5)
-    assert_attention_close(got.view(1, S, heads, HD), ref, "scale 0.5", scaled=True)
+    assert_attention_close(got.view(1, S, heads, HD), ref, "scale 0.5")
 
 
 def test_constant_v_gives_v():
@@ -124,3 +129,45 @@ def test_full_size_workloads_sampled_rows(idx):
     got = oc[torch.from_numpy(rows[:, 0]).cuda(), torch.from_numpy(rows[:, 2]).cuda(),
              torch.from_numpy(rows[:, 1]).cuda()].cpu()
     assert_attention_close(got, ref, w.name)
+
+
+# The 832x480, 81-frame token grid (21, 30, 52): S = 32760, 256 key tiles, the
+# last one ragged (120 keys).
+LONG_S = 32760
+
+
+def _rows_of_head(S, idx):
+    idx = np.asarray(idx, dtype=np.int64)
+    return np.stack([np.zeros_like(idx), np.zeros_like(idx), idx], axis=1)
+
+
+def test_full_length_late_peak_every_row():
+    """Every query equals the key of a token in the last key tile, so each
+    row's running max is set by N(0,1) logits for 255 tiles and jumps by about
+    16 (log2 units) in the last one: the lazy rescale fires there, after the
+    row sum has accumulated 32700 keys, and the peak and the bulk weigh about
+    the same. All 32760 rows of the head against the oracle at the flat bound."""
+    S, heads = LONG_S, 1
+    qkv = wi.packed_qkv(1, S, heads, seed=41)
+    t = torch.randint(S - 60, S, (S,), generator=torch.Generator().manual_seed(42))
+    qkv[0, :, :HD] = qkv[0, t, HD:2 * HD]
+    got = gpu_attention(qkv, heads)
+    ref = oracle.attention_rows(qkv, heads, _rows_of_head(S, np.arange(S)), SCALE)
+    assert_attention_close(got.view(S, HD), ref, "late peak, every row")
+
+
+def test_full_length_rising_max_sampled_rows():
+    """Keys scaled by 2^(4 j / S): each row's tile maxima grow from about 2.5
+    to about 40 (natural-log units) along the 256 tiles, so the running max is
+    raised, and O and the row sum rescaled, every few tiles through the whole
+    loop, and the result is dominated by a few late keys whose weights reach
+    the bf16 rounding of P at its largest. Sampled rows (always the first, the
+    last and the ragged last tile) against the oracle at the flat bound."""
+    S, heads = LONG_S, 1
+    qkv = wi.packed_qkv(1, S, heads, seed=43)
+    g = torch.exp2(4.0 * torch.arange(S, dtype=torch.float32) / S)
+    qkv[0, :, HD:2 * HD] = (qkv[0, :, HD:2 * HD].float() * g[:, None]).to(torch.bfloat16)
+    got = gpu_attention(qkv, heads)
+    idx = wi.sample_rows(S, 4096, seed=44).numpy()
+    ref = oracle.attention_rows(qkv, heads, _rows_of_head(S, idx), SCALE)
+    assert_attention_close(got.view(S, HD)[torch.from_numpy(idx)], ref, "rising max, sampled rows")

@@ -1,10 +1,22 @@
-"""The CUDA side of sequence parallelism on one GPU: N ranks simulated in one
-process, one after another (norm+RoPE of every shard, the gather as a
-concatenation in rank order, attention of every rank's rows -- no kernel waits
-on another), and the single-rank path through sp.cuda_ops; the outputs equal
-the unsharded wan_dit_attn bit for bit."""
+"""The CUDA side of sequence parallelism on one GPU.
+
+All-gather form: N ranks simulated in one process, one after another
+(norm+RoPE of every shard, the gather as a concatenation in rank order,
+attention of every rank's rows -- no kernel waits on another), and the
+single-rank path through sp.cuda_ops; the outputs equal the unsharded
+wan_dit_attn bit for bit, and a shard's rows match the oracle.
+
+Ring form: every rank's rounds run one after another on one GPU, each
+"remote" K|V chunk a local buffer of its own; the partial states and their
+merge match the oracle at the attention bound."""
+import math
+
+import numpy as np
 import pytest
 import torch
+
+import oracle
+from helpers import assert_attention_close
 
 import video_diffusion_transformer_packed_b200 as wan
 import wan_inputs as wi
@@ -82,3 +94,120 @@ def test_shards_starting_mid_row_with_many_batch_boundaries():
     torch.cuda.synchronize()
     assert wan.device_error() == 0
     assert torch.equal(torch.cat(shards, dim=1).view(torch.int16), ref.view(torch.int16))
+
+
+SCALE = 1 / math.sqrt(128)
+LOG2E = 1.4426950408889634
+
+
+def _normed(idx, seed):
+    w = wi.WORKLOADS[idx]
+    qkv, gq, gk = wi.inputs_for(w, seed=seed)
+    d = qkv.cuda()
+    wan.qk_norm_rope(d, w.grid, w.heads, gq.cuda(), gk.cuda())
+    torch.cuda.synchronize()
+    return w, d
+
+
+def _sampled(w, out_rows, rows):
+    """out_rows [B, n, D] (GPU) at (b, h, i) -> [len(rows), 128] on the CPU."""
+    oc = out_rows.view(out_rows.shape[0], out_rows.shape[1], w.heads, 128)
+    r = torch.from_numpy(rows).cuda()
+    return oc[r[:, 0], r[:, 2], r[:, 1]].cpu()
+
+
+def test_shard_rows_match_the_oracle():
+    """wan_self_attention_rows for a rank's shard (rows [3900, 7800) of the
+    5-frame 480p grid) against the oracle's attention of the same rows."""
+    w, d = _normed(1, seed=21)
+    r0, n = 3900, 3900
+    out = wan.self_attention_rows(d, w.heads, r0, n)
+    torch.cuda.synchronize()
+    assert wan.device_error() == 0
+    local = wi.sample_rows(n, 24, seed=22).numpy()
+    rows = np.array([(0, h, i) for h in (0, 17, 39) for i in local], dtype=np.int64)
+    ref = oracle.attention_rows(d.cpu(), w.heads, rows + np.array([0, 0, r0]), SCALE)
+    assert_attention_close(_sampled(w, out, rows), ref, "shard rows")
+
+
+@pytest.mark.parametrize("k0,kn", [(0, 7800), (1000, 1), (129, 3000), (7799, 1), (3900, 3900)])
+def test_partial_state_matches_the_oracle_state(k0, kn):
+    """A key range of the packed buffer: the state's O / l is the attention of
+    that range (flat bound against the oracle's), and its reference max lies
+    within 8 below the range's largest scaled logit (base 2)."""
+    w, d = _normed(1, seed=23)
+    o, ml = wan.self_attention_partial(d, w.heads, d, k_row0=k0, k_rows=kn)
+    torch.cuda.synchronize()
+    assert wan.device_error() == 0
+    local = wi.sample_rows(w.seq_len, 16, seed=24).numpy()
+    rows = np.array([(0, h, i) for h in (0, 39) for i in local], dtype=np.int64)
+    ro, rml = oracle.attention_partial_rows(d.cpu(), w.heads, d.cpu(), k0, kn, rows, SCALE)
+    r = torch.from_numpy(rows).cuda()
+    go = o[r[:, 0], r[:, 2], r[:, 1]].double().cpu().numpy()
+    gml = ml[r[:, 0], r[:, 2], r[:, 1]].double().cpu().numpy()
+    got = torch.from_numpy(go / gml[:, 1:2])
+    assert_attention_close(got, ro / rml[:, 1:2], f"partial [{k0}, {k0 + kn})")
+    m_true = rml[:, 0] * LOG2E
+    assert np.all(gml[:, 0] <= m_true + 1e-3) and np.all(gml[:, 0] >= m_true - 8.0 - 1e-3)
+
+
+@pytest.mark.parametrize("idx,world", [(1, 2), (1, 4), (1, 8), (4, 2), (0, 4)])
+def test_ring_rounds_simulated_on_one_gpu(idx, world):
+    """Every rank's ring rounds, one after another: its own K|V chunk, then
+    its left neighbours' in ring order, each chunk a separate [B, S/N, 2D]
+    buffer; partial states merged round by round and finalised. The union of
+    the ranks' outputs against the oracle on sampled rows of every rank, and
+    against the unsharded kernel."""
+    w, d = _normed(idx, seed=25 + world)
+    S, D = w.seq_len, w.dim
+    if S % world:
+        pytest.skip("sequence not divisible")
+    s_local = S // world
+    shards = [d[:, r * s_local:(r + 1) * s_local].contiguous() for r in range(world)]
+    chunks = [sh[..., D:].contiguous() for sh in shards]
+    outs = []
+    for r in range(world):
+        state = None
+        for c in sp.ring_order(world, r):
+            part = wan.self_attention_partial(shards[r], w.heads, chunks[c])
+            if state is None:
+                state = part
+            else:
+                wan.attention_merge(state[0], state[1], part[0], part[1])
+        outs.append(wan.attention_merge(state[0], state[1], finalize=True))
+    torch.cuda.synchronize()
+    assert wan.device_error() == 0
+    out = torch.cat(outs, dim=1)
+    dense = wan.self_attention(d, w.heads)
+    torch.cuda.synchronize()
+    assert float((out.float() - dense.float()).abs().max()) <= 2e-2
+    local = wi.sample_rows(s_local, 6, seed=26).numpy()
+    idx_rows = np.concatenate([r * s_local + local for r in range(world)])
+    rows = np.array([(b, h, i) for b in range(w.batch) for h in (0, w.heads - 1) for i in idx_rows],
+                    dtype=np.int64)
+    ref = oracle.attention_rows(d.cpu(), w.heads, rows, SCALE)
+    assert_attention_close(_sampled(w, out, rows), ref, f"ring world {world}")
+
+
+def test_ring_and_gather_forms_on_a_side_stream():
+    """Both orchestrations at world size 1 with an explicit non-default
+    stream: every kernel, copy and merge is ordered on that stream, so the
+    results equal the unsharded step's."""
+    w = wi.WORKLOADS[1]
+    qkv, gq, gk = wi.inputs_for(w, seed=27)
+    gq, gk = gq.cuda(), gk.cuda()
+    ref = wan.dit_attn(qkv.cuda(), w.grid, w.heads, gq, gk)
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    a = qkv.cuda()
+    b = qkv.cuda()
+    torch.cuda.synchronize()
+    out_g = sp.sequence_parallel_step(a, w.grid, 1, 0, sp.cuda_ops(w.grid, w.heads, gq, gk, stream=side))
+    out_r = sp.ring_attention_step(b, w.grid, 1, 0, sp.cuda_ring_ops(w.grid, w.heads, gq, gk, stream=side))
+    side.synchronize()
+    assert torch.equal(out_g.view(torch.int16), ref.view(torch.int16))
+    assert float((out_r.float() - ref.float()).abs().max()) <= 2e-2
+    rows = np.array([(0, h, i) for h in (0, 39) for i in wi.sample_rows(w.seq_len, 16, seed=28).tolist()],
+                    dtype=np.int64)
+    normed = oracle.qk_norm_rope(qkv, w.grid, w.heads, gq.cpu(), gk.cpu(), wi.EPS, wi.THETA)
+    assert_attention_close(_sampled(w, out_r, rows), oracle.attention_rows(normed, w.heads, rows, SCALE), "ring")

@@ -29,7 +29,7 @@ THETA = 10000.0
 STATUS = {0: "WAN_OK", 1: "WAN_ERR_NULL", 2: "WAN_ERR_ALIGN", 3: "WAN_ERR_SHAPE",
           4: "WAN_ERR_HEAD_DIM", 5: "WAN_ERR_PARAM", 6: "WAN_ERR_UNSUPPORTED_DEVICE",
           7: "WAN_ERR_LAUNCH", 8: "WAN_ERR_DEVICE_TIMEOUT", 9: "WAN_ERR_ALIAS",
-          10: "WAN_ERR_MEMORY_KIND"}
+          10: "WAN_ERR_MEMORY_KIND", 11: "WAN_ERR_KERNEL_IMAGE"}
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "_lib", "libwanattn.so")
@@ -95,6 +95,11 @@ def load_library() -> ctypes.CDLL:
             lib.wan_qk_norm_rope_shard.restype = I32
             lib.wan_self_attention_rows.argtypes = [P, P, I64, I64, I32, I32, I64, I64, F, P]
             lib.wan_self_attention_rows.restype = I32
+            lib.wan_self_attention_partial.argtypes = [P, I64, I64, I64, P, I64, I64, I64, I64, P, P, I64, I32,
+                                                       I32, F, P]
+            lib.wan_self_attention_partial.restype = I32
+            lib.wan_attention_merge.argtypes = [P, P, P, P, P, I64, I32, P]
+            lib.wan_attention_merge.restype = I32
             _lib = lib
     return _lib
 
@@ -325,6 +330,66 @@ def self_attention_rows(qkv, heads: int, q_row0: int, q_rows: int, out=None, sca
     _check(load_library().wan_self_attention_rows(_bf16_cuda(qkv, "qkv"), _bf16_cuda(out, "out"), B, S, heads,
                                                   HEAD_DIM, int(q_row0), int(q_rows), scale, _stream(stream)),
            "wan_self_attention_rows")
+    return out
+
+
+def _f32_cuda(t, name: str) -> int:
+    import torch
+    if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous():
+        raise TypeError(f"{name} must be a contiguous float32 CUDA tensor")
+    return t.data_ptr()
+
+
+def self_attention_partial(q_qkv, heads: int, kv, q_row0: int = 0, q_rows=None, k_row0: int = 0, k_rows=None,
+                           o=None, ml=None, scale: float = 0.0, stream=None):
+    """Softmax state of query rows [q_row0, q_row0 + q_rows) of the packed
+    q_qkv [B, Sq, 3*heads*128] against keys [k_row0, k_row0 + k_rows) of kv
+    [B, Skv, pitch] (K then V in its last 2*heads*128 columns: a packed QKV
+    buffer or a K|V chunk). Returns (o [B, q_rows, heads, 128] fp32,
+    ml [B, q_rows, heads, 2] fp32): O and (m, l) in base 2."""
+    import torch
+    _check_packed(q_qkv, heads)
+    B, Sq, _ = q_qkv.shape
+    if kv.dim() != 3 or kv.shape[0] != B or kv.shape[2] < 2 * heads * HEAD_DIM:
+        raise ValueError("kv must be [B, Skv, pitch] with K and V in its last 2*heads*128 columns")
+    q_rows = Sq - q_row0 if q_rows is None else q_rows
+    k_rows = kv.shape[1] - k_row0 if k_rows is None else k_rows
+    if o is None:
+        o = torch.empty((B, q_rows, heads, HEAD_DIM), dtype=torch.float32, device=q_qkv.device)
+    if ml is None:
+        ml = torch.empty((B, q_rows, heads, 2), dtype=torch.float32, device=q_qkv.device)
+    if tuple(o.shape) != (B, q_rows, heads, HEAD_DIM) or tuple(ml.shape) != (B, q_rows, heads, 2):
+        raise ValueError("o must be [B, q_rows, heads, 128] and ml [B, q_rows, heads, 2]")
+    _check(load_library().wan_self_attention_partial(
+        _bf16_cuda(q_qkv, "q_qkv"), Sq, int(q_row0), int(q_rows), _bf16_cuda(kv, "kv"), kv.shape[1], kv.shape[2],
+        int(k_row0), int(k_rows), _f32_cuda(o, "o"), _f32_cuda(ml, "ml"), B, heads, HEAD_DIM, scale,
+        _stream(stream)), "wan_self_attention_partial")
+    return o, ml
+
+
+def attention_merge(o_acc, ml_acc, o_part=None, ml_part=None, out=None, finalize: bool = False, stream=None):
+    """(o_acc, ml_acc) := merge with (o_part, ml_part) when given; with
+    finalize, also returns out = bf16(O / l) shaped like o_acc without its last
+    axis split ([B, rows, heads*128] for o_acc [B, rows, heads, 128])."""
+    import torch
+    if o_acc.shape[-1] != HEAD_DIM or tuple(ml_acc.shape) != tuple(o_acc.shape[:-1]) + (2,):
+        raise ValueError("o_acc must be [..., 128] and ml_acc [..., 2] over the same units")
+    if (o_part is None) != (ml_part is None):
+        raise ValueError("o_part and ml_part go together")
+    if o_part is not None and (o_part.shape != o_acc.shape or ml_part.shape != ml_acc.shape):
+        raise ValueError("the partial state must have the accumulator's shape")
+    n_units = o_acc.numel() // HEAD_DIM
+    if finalize and out is None:
+        out = torch.empty(tuple(o_acc.shape[:-2]) + (o_acc.shape[-2] * HEAD_DIM,), dtype=torch.bfloat16,
+                          device=o_acc.device)
+    if out is not None and out.numel() != n_units * HEAD_DIM:
+        raise ValueError("out must hold 128 values per unit")
+    _check(load_library().wan_attention_merge(
+        _f32_cuda(o_acc, "o_acc"), _f32_cuda(ml_acc, "ml_acc"),
+        _f32_cuda(o_part, "o_part") if o_part is not None else None,
+        _f32_cuda(ml_part, "ml_part") if ml_part is not None else None,
+        _bf16_cuda(out, "out") if out is not None else None, n_units, HEAD_DIM, _stream(stream)),
+        "wan_attention_merge")
     return out
 
 

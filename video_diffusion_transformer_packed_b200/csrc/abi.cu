@@ -11,7 +11,7 @@
 
 namespace {
 
-constexpr int32_t kAbiVersion = 8;
+constexpr int32_t kAbiVersion = 9;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -115,6 +115,62 @@ bool overlaps(const void* a, uint64_t na, const void* b, uint64_t nb) {
     if (_s != WAN_OK) return _s; \
   } while (0)
 
+// Status of a plan or launch: a kernel whose compiled register count differs
+// from the one its per-warpgroup register split was written for is refused
+// by the launcher with cudaErrorInvalidKernelImage, and gets its own status.
+int32_t launch_status(cudaError_t e) {
+  if (e == cudaSuccess) return WAN_OK;
+  return e == cudaErrorInvalidKernelImage ? WAN_ERR_KERNEL_IMAGE : WAN_ERR_LAUNCH;
+}
+
+#define WAN_LAUNCH_TRY(expr) WAN_TRY(launch_status(expr))
+
+// The kernels' device error words and the Skip-Softmax counters: one copy of
+// each per device, shared by every launch on that device. They are taken
+// (read and cleared in one atomic exchange each) by a one-thread kernel on
+// the caller's stream, so a word set between the read and the clear cannot be
+// lost; the taken values land in g_taken, which a mutex keeps to one reader
+// at a time.
+struct TakenWords {
+  int attn, norm, fp8, gemm;
+  unsigned long long skip[2];
+};
+__device__ TakenWords g_taken;
+
+__global__ void take_words_kernel(int* attn, int* norm, int* fp8, int* gemm, unsigned long long* skip) {
+  TakenWords t = {0, 0, 0, 0, {0ull, 0ull}};
+  if (attn) t.attn = atomicExch(attn, 0);
+  if (norm) t.norm = atomicExch(norm, 0);
+  if (fp8) t.fp8 = atomicExch(fp8, 0);
+  if (gemm) t.gemm = atomicExch(gemm, 0);
+  if (skip) {
+    t.skip[0] = atomicExch(&skip[0], 0ull);
+    t.skip[1] = atomicExch(&skip[1], 0ull);
+  }
+  g_taken = t;
+}
+
+std::mutex g_take_mutex;
+
+// errors: take the four error words; skip: take the Skip-Softmax counters.
+cudaError_t take_device_words(cudaStream_t stream, bool errors, bool skip, TakenWords* out) {
+  int *attn = nullptr, *norm = nullptr, *fp8 = nullptr, *gemm = nullptr;
+  unsigned long long* skip_stats = nullptr;
+  cudaError_t e = wan::attn_device_words(&attn, &skip_stats);
+  if (e == cudaSuccess && errors) e = wan::norm_error_word(&norm);
+  if (e == cudaSuccess && errors) e = wan::fp8_error_word(&fp8);
+  if (e == cudaSuccess && errors) e = wan::gemm_error_word(&gemm);
+  if (e != cudaSuccess) return e;
+  if (!errors) attn = nullptr;
+  if (!skip) skip_stats = nullptr;
+  std::lock_guard<std::mutex> lock(g_take_mutex);
+  take_words_kernel<<<1, 1, 0, stream>>>(attn, norm, fp8, gemm, skip_stats);
+  e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaMemcpyFromSymbolAsync(out, g_taken, sizeof(TakenWords), 0, cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  return e;
+}
+
 }  // namespace
 
 extern "C" {
@@ -133,6 +189,9 @@ const char* wan_status_string(int32_t status) {
     case WAN_ERR_ALIAS: return "out overlaps qkv";
     case WAN_ERR_MEMORY_KIND:
       return "a host buffer is not page-locked, or a device buffer is not memory of the current device";
+    case WAN_ERR_KERNEL_IMAGE:
+      return "a compiled attention kernel's register count differs from the one its register split was "
+             "written for: rebuild the library with the CUDA toolkit it targets";
     default: return "unknown status";
   }
 }
@@ -163,9 +222,7 @@ int32_t wan_self_attention(const void* qkv, void* out, int64_t batch, int64_t se
   WAN_TRY(check_device());
   (void)cudaGetLastError();
   wan::AttnPlan plan;
-  if (wan::plan_attn_fwd(qkv, out, batch, seq_len, heads, scale, &plan) != cudaSuccess) {
-    return WAN_ERR_LAUNCH;
-  }
+  WAN_LAUNCH_TRY(wan::plan_attn_fwd(qkv, out, batch, seq_len, heads, scale, &plan));
   if (wan::launch_attn_fwd(plan, static_cast<cudaStream_t>(stream), false) != cudaSuccess) {
     return WAN_ERR_LAUNCH;
   }
@@ -178,13 +235,11 @@ int32_t wan_self_attention_sparse(const void* qkv, void* out, int64_t batch, int
   WAN_TRY(check_heads(heads, head_dim));
   WAN_TRY(check_tokens(batch, seq_len, heads));
   WAN_TRY(check_attn_args(qkv, out, batch, seq_len, heads, scale));
-  if (!(std::isfinite(threshold) && threshold >= 0.f)) return WAN_ERR_PARAM;
+  if (!(std::isfinite(threshold) && threshold >= 0.f && threshold <= 1.f)) return WAN_ERR_PARAM;
   WAN_TRY(check_device());
   (void)cudaGetLastError();
   wan::AttnPlan plan;
-  if (wan::plan_attn_fwd(qkv, out, batch, seq_len, heads, scale, &plan) != cudaSuccess) {
-    return WAN_ERR_LAUNCH;
-  }
+  WAN_LAUNCH_TRY(wan::plan_attn_fwd(qkv, out, batch, seq_len, heads, scale, &plan));
   plan.skip_threshold = threshold;
   if (wan::launch_attn_fwd(plan, static_cast<cudaStream_t>(stream), false) != cudaSuccess) {
     return WAN_ERR_LAUNCH;
@@ -256,10 +311,8 @@ int32_t wan_self_attention_fp8(const void* qk8, const void* v8t, void* out, int6
   }
   WAN_TRY(check_device());
   (void)cudaGetLastError();
-  if (wan::launch_attn_fp8(qk8, v8t, out, batch, seq_len, heads, s_pitch, scale, scale_q, scale_k, scale_v,
-                           static_cast<cudaStream_t>(stream)) != cudaSuccess) {
-    return WAN_ERR_LAUNCH;
-  }
+  WAN_LAUNCH_TRY(wan::launch_attn_fp8(qk8, v8t, out, batch, seq_len, heads, s_pitch, scale, scale_q, scale_k,
+                                      scale_v, static_cast<cudaStream_t>(stream)));
   return WAN_OK;
 }
 
@@ -336,20 +389,84 @@ int32_t wan_self_attention_rows(const void* qkv, void* out, int64_t batch, int64
   WAN_TRY(check_device());
   (void)cudaGetLastError();
   wan::AttnPlan plan;
-  if (wan::plan_attn_fwd(qkv, out, batch, seq_len, heads, scale, &plan) != cudaSuccess) return WAN_ERR_LAUNCH;
+  WAN_LAUNCH_TRY(wan::plan_attn_fwd(qkv, out, batch, seq_len, heads, scale, &plan));
   plan.q_row0 = static_cast<int32_t>(q_row0);
   plan.q_rows = static_cast<int32_t>(q_rows);
   if (wan::launch_attn_fwd(plan, static_cast<cudaStream_t>(stream), false) != cudaSuccess) return WAN_ERR_LAUNCH;
   return WAN_OK;
 }
 
-int32_t wan_skip_stats(void* stream, int64_t* group_tiles, int64_t* products) {
-  int64_t g = 0, pr = 0;
-  if (wan::read_and_clear_skip_stats(static_cast<cudaStream_t>(stream), &g, &pr) != cudaSuccess) {
-    return WAN_ERR_LAUNCH;
+int32_t wan_self_attention_partial(const void* q_qkv, int64_t q_seq_len, int64_t q_row0, int64_t q_rows,
+                                   const void* kv, int64_t kv_rows, int64_t kv_pitch, int64_t k_row0,
+                                   int64_t k_rows, float* o, float* ml, int64_t batch, int32_t heads,
+                                   int32_t head_dim, float scale, void* stream) {
+  WAN_TRY(check_heads(heads, head_dim));
+  WAN_TRY(check_tokens(batch, q_seq_len, heads));
+  if (!q_qkv || !kv || !o || !ml) return WAN_ERR_NULL;
+  if (!aligned16(q_qkv) || !aligned16(kv) || !aligned16(o) || !aligned16(ml)) return WAN_ERR_ALIGN;
+  const int64_t d = static_cast<int64_t>(heads) * WAN_HEAD_DIM;
+  if (q_row0 < 0 || q_rows < 1 || q_row0 + q_rows > q_seq_len) return WAN_ERR_SHAPE;
+  if (kv_rows < 1 || kv_rows > INT32_MAX || k_row0 < 0 || k_rows < 1 || k_row0 + k_rows > kv_rows) {
+    return WAN_ERR_SHAPE;
   }
-  if (group_tiles) *group_tiles = g;
-  if (products) *products = pr;
+  // K and V are the last 2D columns of each kv row; rows are whole 16-byte units.
+  if (kv_pitch < 2 * d || kv_pitch % 8 != 0 || kv_pitch > (int64_t)INT32_MAX) return WAN_ERR_SHAPE;
+  if (batch > (INT64_MAX / 4) / (kv_rows * kv_pitch)) return WAN_ERR_SHAPE;
+  if (static_cast<uint64_t>(kv_rows) * static_cast<uint64_t>(kv_pitch) * 2ull >= (1ull << 40)) return WAN_ERR_SHAPE;
+  if (!std::isfinite(scale)) return WAN_ERR_PARAM;
+  const uint64_t q_bytes = static_cast<uint64_t>(batch) * q_seq_len * 3 * d * 2;
+  const uint64_t kv_bytes = static_cast<uint64_t>(batch) * kv_rows * kv_pitch * 2;
+  const uint64_t o_bytes = static_cast<uint64_t>(batch) * q_rows * d * 4;
+  const uint64_t ml_bytes = static_cast<uint64_t>(batch) * q_rows * heads * 8;
+  if (overlaps(o, o_bytes, ml, ml_bytes) || overlaps(o, o_bytes, q_qkv, q_bytes) ||
+      overlaps(o, o_bytes, kv, kv_bytes) || overlaps(ml, ml_bytes, q_qkv, q_bytes) ||
+      overlaps(ml, ml_bytes, kv, kv_bytes)) {
+    return WAN_ERR_ALIAS;
+  }
+  WAN_TRY(check_device());
+  (void)cudaGetLastError();
+  wan::AttnPlan plan;
+  WAN_LAUNCH_TRY(wan::plan_attn_fwd(q_qkv, nullptr, batch, q_seq_len, heads, scale, &plan));
+  WAN_LAUNCH_TRY(wan::plan_attn_kv(kv, batch, kv_rows, kv_pitch, k_row0, k_rows, &plan));
+  plan.q_row0 = static_cast<int32_t>(q_row0);
+  plan.q_rows = static_cast<int32_t>(q_rows);
+  plan.o_part = o;
+  plan.ml_part = ml;
+  WAN_LAUNCH_TRY(wan::launch_attn_fwd(plan, static_cast<cudaStream_t>(stream), false));
+  return WAN_OK;
+}
+
+int32_t wan_attention_merge(float* o_acc, float* ml_acc, const float* o_part, const float* ml_part, void* out,
+                            int64_t n_units, int32_t head_dim, void* stream) {
+  if (head_dim != WAN_HEAD_DIM) return WAN_ERR_HEAD_DIM;
+  if (!o_acc || !ml_acc) return WAN_ERR_NULL;
+  if ((o_part == nullptr) != (ml_part == nullptr) || (o_part == nullptr && out == nullptr)) return WAN_ERR_NULL;
+  if (!aligned16(o_acc) || !aligned16(ml_acc) || (o_part && !aligned16(o_part)) ||
+      (ml_part && !aligned16(ml_part)) || (out && !aligned16(out))) {
+    return WAN_ERR_ALIGN;
+  }
+  if (n_units < 1 || n_units > (INT64_MAX / 1024)) return WAN_ERR_SHAPE;
+  const uint64_t ob = static_cast<uint64_t>(n_units) * WAN_HEAD_DIM * 4, mb = static_cast<uint64_t>(n_units) * 8;
+  const uint64_t yb = static_cast<uint64_t>(n_units) * WAN_HEAD_DIM * 2;
+  if (overlaps(o_acc, ob, ml_acc, mb) ||
+      (o_part && (overlaps(o_part, ob, o_acc, ob) || overlaps(o_part, ob, ml_acc, mb) ||
+                  overlaps(ml_part, mb, o_acc, ob) || overlaps(ml_part, mb, ml_acc, mb))) ||
+      (out && (overlaps(out, yb, o_acc, ob) || overlaps(out, yb, ml_acc, mb) ||
+               (o_part && (overlaps(out, yb, o_part, ob) || overlaps(out, yb, ml_part, mb)))))) {
+    return WAN_ERR_ALIAS;
+  }
+  WAN_TRY(check_device());
+  (void)cudaGetLastError();
+  WAN_LAUNCH_TRY(wan::launch_attn_merge(o_acc, ml_acc, o_part, ml_part, out, n_units,
+                                        static_cast<cudaStream_t>(stream)));
+  return WAN_OK;
+}
+
+int32_t wan_skip_stats(void* stream, int64_t* group_tiles, int64_t* products) {
+  TakenWords t;
+  if (take_device_words(static_cast<cudaStream_t>(stream), false, true, &t) != cudaSuccess) return WAN_ERR_LAUNCH;
+  if (group_tiles) *group_tiles = static_cast<int64_t>(t.skip[0]);
+  if (products) *products = static_cast<int64_t>(t.skip[1]);
   return WAN_OK;
 }
 
@@ -365,9 +482,7 @@ int32_t wan_dit_attn(void* qkv, void* out, int64_t batch, int32_t F, int32_t H, 
   (void)cudaGetLastError();
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   wan::AttnPlan plan;
-  if (wan::plan_attn_fwd(qkv, out, batch, S, heads, scale, &plan) != cudaSuccess) {
-    return WAN_ERR_LAUNCH;
-  }
+  WAN_LAUNCH_TRY(wan::plan_attn_fwd(qkv, out, batch, S, heads, scale, &plan));
   if (wan::launch_qk_norm_rope(qkv, batch, F, H, W, heads, gamma_q, gamma_k, eps, theta, st) !=
       cudaSuccess) {
     return WAN_ERR_LAUNCH;
@@ -414,9 +529,7 @@ int32_t wan_dit_attn_host(const void* qkv_host, void* out_host, void* qkv_dev, v
   step.theta = theta;
   step.scale = scale;
   step.overlap_input = (flags & WAN_HOST_OVERLAP_INPUT) != 0;
-  if (wan::enqueue_dit_attn_host(step, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
-    return WAN_ERR_LAUNCH;
-  }
+  WAN_LAUNCH_TRY(wan::enqueue_dit_attn_host(step, static_cast<cudaStream_t>(stream)));
   return WAN_OK;
 }
 
@@ -429,9 +542,7 @@ int32_t wan_selftest_wait_timeout(const void* qkv, void* out, int64_t batch, int
   WAN_TRY(check_device());
   (void)cudaGetLastError();
   wan::AttnPlan plan;
-  if (wan::plan_attn_fwd(qkv, out, batch, seq_len, heads, 0.f, &plan) != cudaSuccess) {
-    return WAN_ERR_LAUNCH;
-  }
+  WAN_LAUNCH_TRY(wan::plan_attn_fwd(qkv, out, batch, seq_len, heads, 0.f, &plan));
   if (wan::launch_attn_fwd(plan, static_cast<cudaStream_t>(stream), false,
                            static_cast<uint64_t>(wait_limit_ns), true) != cudaSuccess) {
     return WAN_ERR_LAUNCH;
@@ -442,14 +553,9 @@ int32_t wan_selftest_wait_timeout(const void* qkv, void* out, int64_t batch, int
 int32_t wan_device_error(void* stream, int32_t* code) {
   if (!code) return WAN_ERR_NULL;
   *code = 0;
-  int32_t attn = 0, norm = 0, fp8 = 0, gemm = 0;
-  if (wan::read_and_clear_device_error(static_cast<cudaStream_t>(stream), &attn) != cudaSuccess ||
-      wan::read_and_clear_norm_error(static_cast<cudaStream_t>(stream), &norm) != cudaSuccess ||
-      wan::read_and_clear_fp8_error(static_cast<cudaStream_t>(stream), &fp8) != cudaSuccess ||
-      wan::read_and_clear_gemm_error(static_cast<cudaStream_t>(stream), &gemm) != cudaSuccess) {
-    return WAN_ERR_LAUNCH;
-  }
-  *code = attn | (norm << 8) | (fp8 << 16) | ((gemm & 0x7F) << 24);
+  TakenWords t;
+  if (take_device_words(static_cast<cudaStream_t>(stream), true, false, &t) != cudaSuccess) return WAN_ERR_LAUNCH;
+  *code = (t.attn & 0xFF) | ((t.norm & 0xFF) << 8) | ((t.fp8 & 0xFF) << 16) | ((t.gemm & 0x7F) << 24);
   return *code != 0 ? WAN_ERR_DEVICE_TIMEOUT : WAN_OK;
 }
 

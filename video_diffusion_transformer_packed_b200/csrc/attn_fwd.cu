@@ -91,11 +91,15 @@ __device__ unsigned long long g_attn_skip_stats[2];
 
 struct AttnParams {
   uint16_t* out;
-  int32_t S;
+  float* o_part;   // partial mode (not null): fp32 unnormalised O instead of out
+  float* ml_part;  // partial mode: (m, l) of every (row, head)
+  int32_t k_rows;  // keys [k_row0, k_row0 + k_rows) of the K/V map
+  int32_t k_row0;
+  int32_t kv_k0, kv_v0;  // columns of K and V of head 0 in the K/V map
   int32_t heads;
   int32_t D;
-  int32_t q_pairs;  // ceil(S / 256): CTAs per (batch, head)
-  int32_t n_kv;     // ceil(S / 128)
+  int32_t q_pairs;  // ceil(q_rows / 256): CTAs per (batch, head)
+  int32_t n_kv;     // ceil(k_rows / 128)
   int32_t b0, h0, nh;  // this launch covers batches [b0, ...) and heads [h0, h0 + nh)
   int32_t q_row0, q_rows;  // query rows [q_row0, q_row0 + q_rows); out holds q_rows rows per batch
   float skip_log2;     // Skip-Softmax: log2 of the threshold (used by the kSkip kernel only)
@@ -125,11 +129,11 @@ __device__ __forceinline__ void flag_error(volatile int* abort, int site) {
 }
 
 // ---------------------------------------------------------------- producer
-__device__ void run_producer(const CUtensorMap* tmap, const AttnParams& p, uint32_t smem,
-                             Bars bars, volatile int* abort, int* issued, int b, int h, int qp) {
+__device__ void run_producer(const CUtensorMap* tmap, const CUtensorMap* tmap_kv, const AttnParams& p,
+                             uint32_t smem, Bars bars, volatile int* abort, int* issued, int b, int h, int qp) {
   grid_dependency_wait();  // the packed buffer may still be written by the norm kernel
   if (p.skip_loads) return;  // self-test of the bounded waits: nothing will arrive
-  const int xq = h * kHD, xk = p.D + h * kHD, xv = 2 * p.D + h * kHD;
+  const int xq = h * kHD, xk = p.kv_k0 + h * kHD, xv = p.kv_v0 + h * kHD;
   issued[kStages] = 1;  // the Q copies
   mbar_arrive_expect_tx(bars.q_full(), 2 * kTileBytes);
   for (int t = 0; t < 2; ++t) {
@@ -150,10 +154,10 @@ __device__ void run_producer(const CUtensorMap* tmap, const AttnParams& p, uint3
     }
     mbar_arrive_expect_tx(bars.kv_full(slot), kTileBytes);
     const int x = (i & 1) ? xv : xk;
-    const int y = (i >> 1) * kBN;
+    const int y = p.k_row0 + (i >> 1) * kBN;
     const uint32_t dst = smem + kOffKV + slot * kTileBytes;
-    tma_load_3d(dst, tmap, bars.kv_full(slot), x, y, b);
-    tma_load_3d(dst + kBoxBytes, tmap, bars.kv_full(slot), x + 64, y, b);
+    tma_load_3d(dst, tmap_kv, bars.kv_full(slot), x, y, b);
+    tma_load_3d(dst + kBoxBytes, tmap_kv, bars.kv_full(slot), x + 64, y, b);
     issued[slot] = use + 1;
   }
   if (!ok) flag_error(abort, kErrProducer);
@@ -324,7 +328,7 @@ __device__ void run_mma(const AttnParams& p, uint32_t smem, Bars bars, volatile 
 }
 
 // ----------------------------------------------------------------- softmax
-template <bool kSkip>
+template <bool kSkip, bool kPartial>
 __device__ void run_softmax(const AttnParams& p, Bars bars, volatile int* abort, uint32_t tmem,
                             int t, int quarter, int lane, int b, int h, int qp,
                             volatile uint8_t* votes) {
@@ -349,7 +353,7 @@ __device__ void run_softmax(const AttnParams& p, Bars bars, volatile int* abort,
     tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(sr + 64));
     tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(sr + 96));
     tmem_wait_ld();
-    const int rem = p.S - j * kBN;  // valid keys in this tile
+    const int rem = p.k_rows - j * kBN;  // valid keys in this tile
     if (rem < kBN) {
 #pragma unroll
       for (int c = 0; c < 128; ++c) sr[c] = c < rem ? sr[c] : __float_as_uint(-INFINITY);
@@ -414,9 +418,13 @@ __device__ void run_softmax(const AttnParams& p, Bars bars, volatile int* abort,
       tmem_wait_st();
     }
     // p = 2^(s * scale * log2(e) - m), two columns per packed instruction.
+    // The row sum adds the bf16-rounded p that the P V product multiplies, so
+    // that the output is a convex combination of V rows: summing the fp32 p
+    // instead leaves a dominant weight's rounding error (up to 2^-9 of it)
+    // uncorrected in the output.
     const uint64_t sl2_2 = f2(sl2, sl2);
     const uint64_t negm2 = f2(-m_run, -m_run);
-    uint64_t sum2[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};  // 4 chains
+    float sums[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // 8 chains
 #pragma unroll
     for (int part = 0; part < kPParts; ++part) {
       uint32_t pk[kPairsPerPart];
@@ -427,8 +435,8 @@ __device__ void run_softmax(const AttnParams& p, Bars bars, volatile int* abort,
         float x0, x1;
         f2_split(x2, x0, x1);
         const float p0 = ex2(x0), p1 = ex2(x1);
-        sum2[e & 3] = add2(sum2[e & 3], f2(p0, p1));
         pk[e] = pack_bf16x2(p0, p1);
+        add_bf16x2_f32(pk[e], sums[2 * (e & 3)], sums[2 * (e & 3) + 1]);
       }
       if constexpr (kPairsPerPart == 64) {
         tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(pk));
@@ -442,9 +450,7 @@ __device__ void run_softmax(const AttnParams& p, Bars bars, volatile int* abort,
       tc_fence_before();
       mbar_arrive(bars.p_full(t, part));
     }
-    float sum_lo, sum_hi;
-    f2_split(add2(add2(sum2[0], sum2[1]), add2(sum2[2], sum2[3])), sum_lo, sum_hi);
-    l_run += sum_lo + sum_hi;
+    l_run += ((sums[0] + sums[1]) + (sums[2] + sums[3])) + ((sums[4] + sums[5]) + (sums[6] + sums[7]));
   }
   if (kSkip && lane == 0 && n_skipped) atomicAdd(&g_attn_skip_stats[0], n_skipped);
   if (!ok) {
@@ -456,9 +462,29 @@ __device__ void run_softmax(const AttnParams& p, Bars bars, volatile int* abort,
     return;
   }
   tc_fence_after();
-  const float inv_l = 1.f / l_run;
   const int row = (2 * qp + t) * kBM + quarter * 32 + lane;  // within this launch's query rows
-  uint16_t* dst = p.out + (static_cast<int64_t>(b) * p.q_rows + row) * p.D + h * kHD;
+  const int64_t unit = (static_cast<int64_t>(b) * p.q_rows + row) * p.heads + h;
+  if constexpr (kPartial) {
+    // Partial mode: the unnormalised state of this key range, for a merge.
+    float4* dst = reinterpret_cast<float4*>(p.o_part + unit * kHD);
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      uint32_t o[32];
+      tmem_ld32(tO + 32 * c, o);
+      tmem_wait_ld();
+      if (row < p.q_rows) {
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          dst[8 * c + v] = make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
+                                       __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3]));
+        }
+      }
+    }
+    if (row < p.q_rows) reinterpret_cast<float2*>(p.ml_part)[unit] = make_float2(m_run, l_run);
+    return;
+  } else {
+  const float inv_l = 1.f / l_run;
+  uint16_t* dst = p.out + unit * kHD;
 #pragma unroll 1
   for (int c = 0; c < 4; ++c) {
     uint32_t o[32];
@@ -474,11 +500,13 @@ __device__ void run_softmax(const AttnParams& p, Bars bars, volatile int* abort,
       }
     }
   }
+  }
 }
 
-template <bool kSkip>
+template <bool kSkip, bool kPartial>
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ CUtensorMap tmap_kv,
+                    const AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -518,7 +546,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(tmem_holder, kTmemCols);
     tmem_relinquish();
   }
-  if (warp == kLoadWarp && lane == 0) tma_prefetch_desc(&tmap);
+  if (warp == kLoadWarp && lane == 0) {
+    tma_prefetch_desc(&tmap);
+    tma_prefetch_desc(&tmap_kv);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -527,7 +558,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp >= 8) {
     regs_decrease<kCtlRegs>();
     if (warp == kLoadWarp) {
-      if (lane == 0) run_producer(&tmap, p, smem_base, bars, abort, issued, b, h, qp);
+      if (lane == 0) run_producer(&tmap, &tmap_kv, p, smem_base, bars, abort, issued, b, h, qp);
     } else if (warp == kMmaWarp) {
       if (lane == 0) {
         run_mma<kSkip>(p, smem_base, bars, abort, tmem, reinterpret_cast<const volatile uint32_t*>(votes));
@@ -536,7 +567,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     regs_increase<kSoftmaxRegs>();
-    run_softmax<kSkip>(p, bars, abort, tmem, warp >> 2, warp & 3, lane, b, h, qp, votes);
+    run_softmax<kSkip, kPartial>(p, bars, abort, tmem, warp >> 2, warp & 3, lane, b, h, qp, votes);
   }
 
   tc_fence_before();
@@ -563,21 +594,40 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   return fn;
 }
 
+
+// A 3D tensor map over a [batch][rows][pitch] bf16 buffer: x = channel,
+// y = token, z = batch. Boxes are 64 channels (128 bytes, the swizzle span) x
+// 128 tokens; rows past `rows` read as zeros within the batch element.
+cudaError_t encode_rows_map(void* map, const void* base, int64_t pitch, int64_t rows, int64_t batch) {
+  auto encode = get_encode_fn();
+  if (!encode) return cudaErrorNotSupported;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(pitch), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(batch)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(pitch) * 2,
+                           static_cast<cuuint64_t>(pitch) * 2 * static_cast<cuuint64_t>(rows)};
+  cuuint32_t box[3] = {64, kBM, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = encode(reinterpret_cast<CUtensorMap*>(map), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                      const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 }  // namespace
 
 cudaError_t plan_attn_fwd(const void* qkv, void* out, int64_t batch, int64_t seq_len,
                           int32_t heads, float scale, AttnPlan* plan) {
   static_assert(sizeof(CUtensorMap) == sizeof(plan->tmap), "tensor map size");
+  static_assert(sizeof(CUtensorMap) == sizeof(plan->tmap_kv), "tensor map size");
   const int32_t S = static_cast<int32_t>(seq_len);
   const int32_t D = heads * kHD;
-  auto encode = get_encode_fn();
-  if (!encode) return cudaErrorNotSupported;
 
   static PerDeviceOnce setup;
   const cudaError_t attr_err = setup.run([](int) {
     // The register split inside the kernel is only safe when the compiled
     // kernel launches with exactly kLaunchRegs registers per thread.
-    for (auto kernel : {attn_fwd_kernel<false>, attn_fwd_kernel<true>}) {
+    for (auto kernel : {attn_fwd_kernel<false, false>, attn_fwd_kernel<true, false>, attn_fwd_kernel<false, true>}) {
       cudaFuncAttributes fa;
       cudaError_t e = cudaFuncGetAttributes(&fa, kernel);
       if (e == cudaSuccess && fa.numRegs != kLaunchRegs) e = cudaErrorInvalidKernelImage;
@@ -588,19 +638,10 @@ cudaError_t plan_attn_fwd(const void* qkv, void* out, int64_t batch, int64_t seq
   });
   if (attr_err != cudaSuccess) return attr_err;
 
-  // Packed buffer as a 3D tensor: x = channel (3D), y = token, z = batch.
-  // Boxes are 64 channels (128 bytes, the swizzle span) x 128 tokens.
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(3 * D), static_cast<cuuint64_t>(S),
-                        static_cast<cuuint64_t>(batch)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(3 * D) * 2,
-                           static_cast<cuuint64_t>(3 * D) * 2 * static_cast<cuuint64_t>(S)};
-  cuuint32_t box[3] = {64, kBM, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = encode(reinterpret_cast<CUtensorMap*>(plan->tmap), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
-                      const_cast<void*>(qkv), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  // Q, K and V all come from the packed buffer: one map serves both roles.
+  const cudaError_t e = encode_rows_map(plan->tmap, qkv, 3 * static_cast<int64_t>(D), S, batch);
+  if (e != cudaSuccess) return e;
+  memcpy(plan->tmap_kv, plan->tmap, sizeof(plan->tmap));
 
   plan->out = out;
   plan->S = S;
@@ -617,6 +658,29 @@ cudaError_t plan_attn_fwd(const void* qkv, void* out, int64_t batch, int64_t seq
   plan->nb = static_cast<int32_t>(batch);
   plan->h0 = 0;
   plan->nh = heads;
+  plan->k_row0 = 0;
+  plan->k_rows = S;
+  plan->kv_k0 = D;
+  plan->kv_v0 = 2 * D;
+  plan->o_part = nullptr;
+  plan->ml_part = nullptr;
+  return cudaSuccess;
+}
+
+cudaError_t plan_attn_kv(const void* kv, int64_t batch, int64_t kv_rows, int64_t pitch, int64_t k_row0,
+                         int64_t k_rows, AttnPlan* plan) {
+  const int64_t D = plan->D;
+  if (pitch < 2 * D || pitch % 8 != 0 || k_row0 < 0 || k_rows < 1 || k_row0 + k_rows > kv_rows ||
+      kv_rows > INT32_MAX) {
+    return cudaErrorInvalidValue;
+  }
+  const cudaError_t e = encode_rows_map(plan->tmap_kv, kv, pitch, kv_rows, batch);
+  if (e != cudaSuccess) return e;
+  plan->k_row0 = static_cast<int32_t>(k_row0);
+  plan->k_rows = static_cast<int32_t>(k_rows);
+  plan->kv_k0 = static_cast<int32_t>(pitch - 2 * D);
+  plan->kv_v0 = static_cast<int32_t>(pitch - D);
+  plan->n_kv = static_cast<int32_t>((k_rows + kBN - 1) / kBN);
   return cudaSuccess;
 }
 
@@ -624,7 +688,12 @@ cudaError_t launch_attn_fwd(const AttnPlan& plan, cudaStream_t stream, bool pdl,
                             bool skip_loads) {
   AttnParams p;
   p.out = static_cast<uint16_t*>(plan.out);
-  p.S = plan.S;
+  p.o_part = plan.o_part;
+  p.ml_part = plan.ml_part;
+  p.k_rows = plan.k_rows;
+  p.k_row0 = plan.k_row0;
+  p.kv_k0 = plan.kv_k0;
+  p.kv_v0 = plan.kv_v0;
   p.heads = plan.heads;
   p.D = plan.D;
   p.n_kv = plan.n_kv;
@@ -638,14 +707,17 @@ cudaError_t launch_attn_fwd(const AttnPlan& plan, cudaStream_t stream, bool pdl,
   p.skip_log2 = plan.skip_threshold > 0.f ? log2f(plan.skip_threshold) : -INFINITY;
   p.wait_ns = wait_ns;
   p.skip_loads = skip_loads ? 1 : 0;
-  CUtensorMap tmap;
+  CUtensorMap tmap, tmap_kv;
   memcpy(&tmap, plan.tmap, sizeof(tmap));
+  memcpy(&tmap_kv, plan.tmap_kv, sizeof(tmap_kv));
 
   cudaLaunchConfig_t cfg = {};
   const int64_t grid = static_cast<int64_t>(plan.nb) * plan.nh * p.q_pairs;
   if (plan.nb < 1 || plan.nh < 1 || plan.h0 < 0 || plan.b0 < 0 || plan.h0 + plan.nh > plan.heads ||
       plan.q_row0 < 0 || plan.q_rows < 1 || static_cast<int64_t>(plan.q_row0) + plan.q_rows > plan.S ||
-      grid > INT32_MAX) {
+      plan.k_row0 < 0 || plan.k_rows < 1 || plan.n_kv != (plan.k_rows + kBN - 1) / kBN ||
+      (plan.o_part != nullptr) != (plan.ml_part != nullptr) ||
+      (plan.o_part != nullptr && plan.skip_threshold > 0.f) || grid > INT32_MAX) {
     return cudaErrorInvalidValue;
   }
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
@@ -657,37 +729,16 @@ cudaError_t launch_attn_fwd(const AttnPlan& plan, cudaStream_t stream, bool pdl,
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  if (plan.skip_threshold > 0.f) return cudaLaunchKernelEx(&cfg, attn_fwd_kernel<true>, tmap, p);
-  return cudaLaunchKernelEx(&cfg, attn_fwd_kernel<false>, tmap, p);
+  if (plan.skip_threshold > 0.f) return cudaLaunchKernelEx(&cfg, attn_fwd_kernel<true, false>, tmap, tmap_kv, p);
+  if (plan.o_part != nullptr) return cudaLaunchKernelEx(&cfg, attn_fwd_kernel<false, true>, tmap, tmap_kv, p);
+  return cudaLaunchKernelEx(&cfg, attn_fwd_kernel<false, false>, tmap, tmap_kv, p);
 }
 
-cudaError_t read_and_clear_skip_stats(cudaStream_t stream, int64_t* group_tiles, int64_t* products) {
-  cudaError_t e = cudaStreamSynchronize(stream);
+cudaError_t attn_device_words(int** error_word, unsigned long long** skip_stats) {
+  cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(error_word), g_attn_error_word);
   if (e != cudaSuccess) return e;
-  unsigned long long v[2] = {0, 0};
-  e = cudaMemcpyFromSymbol(v, g_attn_skip_stats, sizeof(v));
-  if (e != cudaSuccess) return e;
-  const unsigned long long zero[2] = {0, 0};
-  e = cudaMemcpyToSymbol(g_attn_skip_stats, zero, sizeof(zero));
-  if (e != cudaSuccess) return e;
-  *group_tiles = static_cast<int64_t>(v[0]);
-  *products = static_cast<int64_t>(v[1]);
-  return cudaSuccess;
+  return cudaGetSymbolAddress(reinterpret_cast<void**>(skip_stats), g_attn_skip_stats);
 }
 
-cudaError_t read_and_clear_device_error(cudaStream_t stream, int32_t* code) {
-  cudaError_t e = cudaStreamSynchronize(stream);
-  if (e != cudaSuccess) return e;
-  int v = 0;
-  e = cudaMemcpyFromSymbol(&v, g_attn_error_word, sizeof(int));
-  if (e != cudaSuccess) return e;
-  if (v != 0) {
-    const int zero = 0;
-    e = cudaMemcpyToSymbol(g_attn_error_word, &zero, sizeof(int));
-    if (e != cudaSuccess) return e;
-  }
-  *code = v;
-  return cudaSuccess;
-}
 
 }  // namespace wan

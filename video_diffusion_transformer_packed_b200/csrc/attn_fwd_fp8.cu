@@ -543,19 +543,8 @@ cudaError_t launch_attn_fp8(const void* qk8, const void* v8t, void* out, int64_t
   return cudaLaunchKernelEx(&cfg, attn_fwd_fp8_kernel, map_qk, map_v, p);
 }
 
-cudaError_t read_and_clear_fp8_error(cudaStream_t stream, int32_t* code) {
-  cudaError_t e = cudaStreamSynchronize(stream);
-  if (e != cudaSuccess) return e;
-  int v = 0;
-  e = cudaMemcpyFromSymbol(&v, g_attn_fp8_error_word, sizeof(int));
-  if (e != cudaSuccess) return e;
-  if (v != 0) {
-    const int zero = 0;
-    e = cudaMemcpyToSymbol(g_attn_fp8_error_word, &zero, sizeof(int));
-    if (e != cudaSuccess) return e;
-  }
-  *code = v;
-  return cudaSuccess;
+cudaError_t fp8_error_word(int** word) {
+  return cudaGetSymbolAddress(reinterpret_cast<void**>(word), g_attn_fp8_error_word);
 }
 
 }  // namespace wan

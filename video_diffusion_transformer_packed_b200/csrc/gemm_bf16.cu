@@ -355,19 +355,8 @@ cudaError_t launch_gemm_bf16(const void* x, const void* w, void* y, int64_t M, i
   return cudaLaunchKernelEx(&cfg, gemm_bf16_kernel, map_x, map_w, p);
 }
 
-cudaError_t read_and_clear_gemm_error(cudaStream_t stream, int32_t* code) {
-  cudaError_t e = cudaStreamSynchronize(stream);
-  if (e != cudaSuccess) return e;
-  int v = 0;
-  e = cudaMemcpyFromSymbol(&v, g_gemm_error_word, sizeof(int));
-  if (e != cudaSuccess) return e;
-  if (v != 0) {
-    const int zero = 0;
-    e = cudaMemcpyToSymbol(g_gemm_error_word, &zero, sizeof(int));
-    if (e != cudaSuccess) return e;
-  }
-  *code = v;
-  return cudaSuccess;
+cudaError_t gemm_error_word(int** word) {
+  return cudaGetSymbolAddress(reinterpret_cast<void**>(word), g_gemm_error_word);
 }
 
 }  // namespace wan

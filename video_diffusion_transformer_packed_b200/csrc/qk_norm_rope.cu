@@ -583,19 +583,8 @@ cudaError_t launch_qk_norm_rope(void* qkv, int64_t batch, int32_t F, int32_t H, 
   return launch_vpt_dispatch<false>(vpt, p, smem_bytes, stream);
 }
 
-cudaError_t read_and_clear_norm_error(cudaStream_t stream, int32_t* code) {
-  cudaError_t e = cudaStreamSynchronize(stream);
-  if (e != cudaSuccess) return e;
-  int v = 0;
-  e = cudaMemcpyFromSymbol(&v, g_norm_error_word, sizeof(int));
-  if (e != cudaSuccess) return e;
-  if (v != 0) {
-    const int zero = 0;
-    e = cudaMemcpyToSymbol(g_norm_error_word, &zero, sizeof(int));
-    if (e != cudaSuccess) return e;
-  }
-  *code = v;
-  return cudaSuccess;
+cudaError_t norm_error_word(int** word) {
+  return cudaGetSymbolAddress(reinterpret_cast<void**>(word), g_norm_error_word);
 }
 
 }  // namespace wan

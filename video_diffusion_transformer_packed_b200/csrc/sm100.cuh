@@ -350,6 +350,16 @@ __device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
   return r;
 }
+// lo_acc += low bf16 of pk, hi_acc += high bf16 of pk, each a mixed-precision
+// fp32 add of the exact bf16 value (no separate conversion).
+__device__ __forceinline__ void add_bf16x2_f32(uint32_t pk, float& lo_acc, float& hi_acc) {
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "mov.b32 {lo, hi}, %2;\n\t"
+      "add.rn.f32.bf16 %0, lo, %0;\n\t"
+      "add.rn.f32.bf16 %1, hi, %1;\n\t}"
+      : "+f"(lo_acc), "+f"(hi_acc)
+      : "r"(pk));
+}
 // max(a, b, c) in one instruction.
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float r;

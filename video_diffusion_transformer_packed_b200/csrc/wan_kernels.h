@@ -45,7 +45,8 @@ cudaError_t launch_qk_norm_rope(void* qkv, int64_t batch, int32_t F, int32_t H, 
 // launched (tensor-map encoding can fail; a launch after a successful plan
 // only fails if the runtime rejects it).
 struct AttnPlan {
-  alignas(64) unsigned char tmap[128];  // CUtensorMap over the packed buffer
+  alignas(64) unsigned char tmap[128];     // CUtensorMap over the buffer holding Q
+  alignas(64) unsigned char tmap_kv[128];  // CUtensorMap over the buffer holding K and V
   void* out;
   int32_t S, heads, D, q_pairs, n_kv;
   float scale_log2;
@@ -55,13 +56,37 @@ struct AttnPlan {
   int32_t b0, nb, h0, nh;
   // Skip-Softmax threshold (0 = dense; plan_attn_fwd sets 0).
   float skip_threshold;
-  // Query rows [q_row0, q_row0 + q_rows) of every batch element attend all S
-  // keys; out holds q_rows rows per batch element (plan_attn_fwd: 0 and S).
+  // Query rows [q_row0, q_row0 + q_rows) of every batch element; out holds
+  // q_rows rows per batch element (plan_attn_fwd: 0 and S).
   int32_t q_row0, q_rows;
+  // Keys [k_row0, k_row0 + k_rows) of the K/V buffer; K of head h at column
+  // kv_k0 + 128 h, V at kv_v0 + 128 h (plan_attn_fwd: the packed buffer
+  // itself, 0, S, D, 2D; plan_attn_kv points them elsewhere).
+  int32_t k_row0, k_rows, kv_k0, kv_v0;
+  // Partial mode (o_part not null): instead of out, the launch writes the
+  // unnormalised fp32 O to o_part [batch][q_rows][heads][128] and (m, l) to
+  // ml_part [batch][q_rows][heads][2], with O = sum_j 2^(a_j - m) v_j and
+  // l = sum_j 2^(a_j - m) over the key range, a_j = scale log2(e) q . k_j.
+  float* o_part;
+  float* ml_part;
 };
 
 cudaError_t plan_attn_fwd(const void* qkv, void* out, int64_t batch, int64_t seq_len,
                           int32_t heads, float scale, AttnPlan* plan);
+
+// Points a plan's K/V source at another buffer: kv is [batch][kv_rows][pitch]
+// bf16 with K and V in its last 2*heads*128 columns (pitch = 3D for a packed
+// QKV buffer, 2D for a K|V buffer); the keys are rows [k_row0, k_row0 + k_rows).
+cudaError_t plan_attn_kv(const void* kv, int64_t batch, int64_t kv_rows, int64_t pitch, int64_t k_row0,
+                         int64_t k_rows, AttnPlan* plan);
+
+// Merges partial attention states (attn_merge.cu): for each of n_units
+// (row, head) units, (o_acc, ml_acc) := the log-sum-exp combination of itself
+// and (o_part, ml_part) when o_part is not null; then, when out is not null,
+// out = bf16(o_acc / l_acc). Layouts as AttnPlan's partial mode (o: 128 floats
+// per unit, ml: 2 floats per unit); out: 128 bf16 per unit.
+cudaError_t launch_attn_merge(float* o_acc, float* ml_acc, const float* o_part, const float* ml_part,
+                              void* out, int64_t n_units, cudaStream_t stream);
 
 // Flash attention over the packed buffer. `pdl` marks the launch as a
 // programmatic dependent of the previous kernel on the stream; `wait_ns`
@@ -100,7 +125,6 @@ cudaError_t launch_qkv_amax(const void* qkv, int64_t tokens, int32_t heads, floa
 cudaError_t launch_attn_fp8(const void* qk8, const void* v8t, void* out, int64_t batch, int64_t seq_len,
                             int32_t heads, int64_t s_pitch, float scale, float scale_q, float scale_k,
                             float scale_v, cudaStream_t stream);
-cudaError_t read_and_clear_fp8_error(cudaStream_t stream, int32_t* code);
 
 // Y[M][N] = X[M][K] W[N][K]^T in bf16 with fp32 accumulation (gemm_bf16.cu);
 // N a multiple of 256, K of 64. When stats is not null, stats[row][j] (row
@@ -108,14 +132,15 @@ cudaError_t read_and_clear_fp8_error(cudaStream_t stream, int32_t* code);
 // of row `row` in columns [256 j, 256 j + 256), for j < stat_cols / 256.
 cudaError_t launch_gemm_bf16(const void* x, const void* w, void* y, int64_t M, int64_t N, int64_t K,
                              double* stats, int64_t stat_cols, cudaStream_t stream);
-cudaError_t read_and_clear_gemm_error(cudaStream_t stream, int32_t* code);
 
-// Synchronise the stream, then read and clear the Skip-Softmax counters:
-// (32-row group, key tile) pairs skipped, and P V products skipped.
-cudaError_t read_and_clear_skip_stats(cudaStream_t stream, int64_t* group_tiles, int64_t* products);
-
-// Synchronise the stream, then read and clear a kernel's device error word.
-cudaError_t read_and_clear_device_error(cudaStream_t stream, int32_t* code);
-cudaError_t read_and_clear_norm_error(cudaStream_t stream, int32_t* code);
+// Device addresses (on the current device) of the words the kernels set when
+// a bounded wait gives up, and of the Skip-Softmax counters ([0] (32-row
+// group, key tile) pairs skipped, [1] P V products skipped). One copy of each
+// per device, shared by every launch; the ABI takes and clears them
+// atomically on the caller's stream.
+cudaError_t attn_device_words(int** error_word, unsigned long long** skip_stats);
+cudaError_t norm_error_word(int** word);
+cudaError_t fp8_error_word(int** word);
+cudaError_t gemm_error_word(int** word);
 
 }  // namespace wan

@@ -17,7 +17,7 @@ import oracle
 import video_diffusion_transformer_packed_b200 as wan
 import wan_inputs as wi
 from video_diffusion_transformer_packed_b200 import build as wan_build
-from helpers import bf16_ulp_distance
+from helpers import assert_attention_close, bf16_ulp_distance
 
 pytestmark = pytest.mark.gpu
 
@@ -100,3 +100,57 @@ def test_qkv_projection_full_size_sampled_rows():
     ref = (yv[:, :2 * D] ** 2).reshape(len(rows), 2 * D // 256, 256).sum(axis=2)
     np.testing.assert_allclose(stats[torch.as_tensor(rows).cuda()].cpu().numpy(), ref, rtol=1e-12,
                                atol=256 * 2.0 ** -126)
+
+
+@pytest.mark.parametrize("name", ["tiny_5x8x8_h12_b1", "a14b_480p_81f_cfg_b2"])
+def test_block_chain_against_the_oracle_chain(name):
+    """The DiT block's self-attention from activations to the output
+    projection, all on the GPU through the C ABI:
+        wan_linear (QKV projection, with the norm's statistic)
+        -> wan_qk_norm_rope_stats -> wan_self_attention
+        -> wan_linear (output projection, tokens x D -> D),
+    against the oracle's chain from the same activations and weights:
+        linear_bf16 -> qk_norm_rope -> attention_rows (rounded to bf16, the
+        output's storage type) -> linear_rows,
+    on sampled tokens (every token of the tiny grid; at the bench shape the
+    first, the last, the ragged last tile and random ones), every output
+    channel, at the attention bar. Each stage is also checked on the GPU's
+    own input to it, so that a failure names its stage."""
+    w_ = wi.BY_NAME[name]
+    B, S, D, heads = w_.batch, w_.seq_len, w_.dim, w_.heads
+    g = torch.Generator().manual_seed(71)
+    x = torch.randn(B * S, D, generator=g).to(torch.bfloat16)
+    wqkv = (torch.randn(3 * D, D, generator=g) / D ** 0.5).to(torch.bfloat16)
+    wo = (torch.randn(D, D, generator=g) / D ** 0.5).to(torch.bfloat16)
+    gq, gk = wi.gammas(heads)
+    # GPU chain
+    qkv, stats = wan.linear(x.cuda(), wqkv.cuda(), stat_cols=2 * D)
+    qkv = qkv.view(B, S, 3 * D)
+    proj = qkv.cpu()
+    wan.qk_norm_rope_stats(qkv, w_.grid, heads, gq.cuda(), gk.cuda(), stats)
+    normed = qkv.cpu()
+    attn = wan.self_attention(qkv, heads)
+    y, _ = wan.linear(attn.view(B * S, D), wo.cuda())
+    torch.cuda.synchronize()
+    assert wan.device_error() == 0
+    attn_h = attn.cpu().view(B * S, D)
+    if S <= 4096:
+        toks = np.arange(B * S)
+    else:
+        local = wi.sample_rows(S, 20, seed=72).numpy()
+        toks = np.concatenate([b * S + local for b in range(B)])
+    # stage by stage, each on the GPU's own input
+    _check_rows(proj.view(B * S, 3 * D), x, wqkv, toks)
+    tk = np.stack([toks // S, toks % S], axis=1)
+    nr = oracle.qk_norm_rope_tokens(proj, w_.grid, heads, gq, gk, wi.EPS, wi.THETA, tk)
+    assert int(bf16_ulp_distance(normed.view(B * S, 3 * D)[torch.from_numpy(toks), :2 * D], nr).max()) <= 1
+    rows = np.array([(t // S, h, t % S) for t in toks for h in range(heads)], dtype=np.int64)
+    a_ref = oracle.attention_rows(normed, heads, rows, 1 / 128 ** 0.5)
+    assert_attention_close(attn_h[torch.from_numpy(toks)].view(-1, 128), a_ref, f"{name}: attention stage")
+    _check_rows(y.cpu(), attn_h, wo, toks)
+    # the oracle's own chain from the activations
+    o_proj = oracle.linear_bf16(x, wqkv).view(B, S, 3 * D)
+    o_normed = oracle.qk_norm_rope(o_proj, w_.grid, heads, gq, gk, wi.EPS, wi.THETA)
+    o_attn = oracle.to_bf16(oracle.attention_rows(o_normed, heads, rows, 1 / 128 ** 0.5)).view(len(toks), D)
+    o_y = oracle.linear_rows(o_attn, wo, np.arange(len(toks)))
+    assert_attention_close(y.cpu()[torch.from_numpy(toks)], o_y, f"{name}: chain output")

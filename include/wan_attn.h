@@ -75,9 +75,11 @@ typedef enum {
   WAN_ERR_ALIAS = 9,              /* out overlaps qkv */
   WAN_ERR_MEMORY_KIND = 10,       /* a host buffer is not page-locked, or a device buffer
                                      is not memory of the current device */
-  WAN_ERR_KERNEL_IMAGE = 11       /* a compiled attention kernel's register count differs from
+  WAN_ERR_KERNEL_IMAGE = 11,      /* a compiled attention kernel's register count differs from
                                      the one its per-warpgroup register split was written for
                                      (a toolkit other than the one the library targets) */
+  WAN_ERR_TOO_LARGE = 12          /* the step does not fit wan_dit_attn_host_static's device
+                                     buffer (WAN_HOST_STATIC_MAX_ELEMENTS) */
 } wan_status;
 
 /* wan_dit_attn_host flag: the call does not wait for earlier work on
@@ -339,6 +341,57 @@ WAN_API int32_t wan_dit_attn_host(const void* qkv_host, void* out_host, void* qk
                                   int32_t head_dim, const void* gamma_q, const void* gamma_k,
                                   float eps, float theta, float scale, int32_t heads_per_chunk,
                                   int32_t flags, void* stream);
+
+/* Largest batch * F*H*W * heads * 128 that wan_dit_attn_host_static takes:
+ * its device buffer holds 8 bytes per element (packed QKV, 6, and the
+ * output, 2), 64 MiB in all. */
+#define WAN_HOST_STATIC_MAX_ELEMENTS (8 * 1024 * 1024)
+
+/*
+ * wan_dit_attn_host for callers that cannot allocate device memory. This
+ * entry point has no counterpart on the pages; it is the host-buffer step
+ * with its device staging in memory the library owns.
+ *
+ * Why: some callers have no way to get device memory for the staging buffers
+ * that wan_dit_attn_host asks for. One example is a host application that
+ * hands this library only host buffers and owns no device allocator. Another
+ * is a process whose device memory is reserved by another runtime's pool,
+ * where cudaMalloc would fail. A third is a latency-bound caller that cannot
+ * afford cudaMalloc's implicit device-wide synchronisation. This call
+ * allocates nothing: no cudaMalloc, no cudaFree, no allocating library
+ * routine.
+ *
+ * The staging is a fixed array of device memory inside the library,
+ * 8 * WAN_HOST_STATIC_MAX_ELEMENTS bytes (64 MiB). Every GPU that loads the
+ * library holds its copy of the array until the process exits.
+ * batch * F*H*W * heads * 128 above WAN_HOST_STATIC_MAX_ELEMENTS returns
+ * WAN_ERR_TOO_LARGE before anything is launched.
+ *
+ * The first call on a device looks up the array's device address, with that
+ * device current. The first call also creates the pipeline's internal
+ * streams and events, as wan_dit_attn_host's first call does. Make that first
+ * call on each device before any stream capture.
+ *
+ * Every call uses the same array, and the array keeps the last call's
+ * contents: its packed QKV after norm+RoPE, and its output. Nothing in the
+ * array has to start at zero, because each call overwrites what it reads.
+ * Two calls that used the array at the same time on the GPU would overwrite
+ * each other's data, so they must not overlap there. The library keeps them
+ * apart: each call's copies and kernels wait for the previous call's use of
+ * the array, through the same per-buffer ordering that wan_dit_attn_host
+ * applies to a reused pair of device buffers. Calls from several host
+ * threads or streams are therefore serialised on the device, and
+ * WAN_HOST_OVERLAP_INPUT gains no overlap here.
+ *
+ * Arguments, layouts, execution and errors are those of wan_dit_attn_host
+ * without qkv_dev and out_dev. qkv_host and out_host are page-locked host
+ * memory (WAN_ERR_MEMORY_KIND otherwise). gamma_q and gamma_k are device
+ * pointers, as before.
+ */
+WAN_API int32_t wan_dit_attn_host_static(const void* qkv_host, void* out_host, int64_t batch, int32_t F, int32_t H,
+                                         int32_t W, int32_t heads, int32_t head_dim, const void* gamma_q,
+                                         const void* gamma_k, float eps, float theta, float scale,
+                                         int32_t heads_per_chunk, int32_t flags, void* stream);
 
 /*
  * Reads and clears the device-side error words that the kernels set when one

@@ -29,7 +29,7 @@ THETA = 10000.0
 STATUS = {0: "WAN_OK", 1: "WAN_ERR_NULL", 2: "WAN_ERR_ALIGN", 3: "WAN_ERR_SHAPE",
           4: "WAN_ERR_HEAD_DIM", 5: "WAN_ERR_PARAM", 6: "WAN_ERR_UNSUPPORTED_DEVICE",
           7: "WAN_ERR_LAUNCH", 8: "WAN_ERR_DEVICE_TIMEOUT", 9: "WAN_ERR_ALIAS",
-          10: "WAN_ERR_MEMORY_KIND", 11: "WAN_ERR_KERNEL_IMAGE"}
+          10: "WAN_ERR_MEMORY_KIND", 11: "WAN_ERR_KERNEL_IMAGE", 12: "WAN_ERR_TOO_LARGE"}
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "_lib", "libwanattn.so")
@@ -100,6 +100,8 @@ def load_library() -> ctypes.CDLL:
             lib.wan_self_attention_partial.restype = I32
             lib.wan_attention_merge.argtypes = [P, P, P, P, P, I64, I32, P]
             lib.wan_attention_merge.restype = I32
+            lib.wan_dit_attn_host_static.argtypes = [P, P, I64, I32, I32, I32, I32, I32, P, P, F, F, F, I32, I32, P]
+            lib.wan_dit_attn_host_static.restype = I32
             _lib = lib
     return _lib
 
@@ -457,6 +459,31 @@ def dit_attn_host(qkv_host, grid: Sequence[int], heads: int, gamma_q, gamma_k, o
                                             _bf16_cuda(gamma_k, "gamma_k"), eps, theta, scale,
                                             int(heads_per_chunk), 1 if overlap_input else 0, _stream(stream)),
            "wan_dit_attn_host")
+    return out_host
+
+
+def dit_attn_host_static(qkv_host, grid: Sequence[int], heads: int, gamma_q, gamma_k, out_host=None,
+                         heads_per_chunk: int = 0, eps: float = EPS, theta: float = THETA, scale: float = 0.0,
+                         overlap_input: bool = False, stream=None):
+    """dit_attn_host through the library's own device buffer instead of caller
+    buffers (for callers that cannot allocate device memory): nothing is
+    allocated on the device; batch * S * heads * 128 must not exceed
+    WAN_HOST_STATIC_MAX_ELEMENTS (8 Mi). Asynchronous on `stream`."""
+    import torch
+    F, H, W = grid
+    _check_packed(qkv_host, heads, grid)
+    _check_gamma(gamma_q, heads, "gamma_q")
+    _check_gamma(gamma_k, heads, "gamma_k")
+    B, S, _ = qkv_host.shape
+    if out_host is None:
+        out_host = torch.empty((B, S, heads * HEAD_DIM), dtype=torch.bfloat16).pin_memory()
+    _check_out(out_host, qkv_host, heads)
+    _check(load_library().wan_dit_attn_host_static(_bf16_pinned(qkv_host, "qkv_host"),
+                                                   _bf16_pinned(out_host, "out_host"), B, F, H, W, heads,
+                                                   HEAD_DIM, _bf16_cuda(gamma_q, "gamma_q"),
+                                                   _bf16_cuda(gamma_k, "gamma_k"), eps, theta, scale,
+                                                   int(heads_per_chunk), 1 if overlap_input else 0,
+                                                   _stream(stream)), "wan_dit_attn_host_static")
     return out_host
 
 

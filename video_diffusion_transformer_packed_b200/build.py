@@ -17,7 +17,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 SOURCES = ["abi.cu", "qk_norm_rope.cu", "attn_fwd.cu", "host_pipeline.cu", "fp8_quant.cu", "attn_fwd_fp8.cu", "gemm_bf16.cu",
-           "attn_merge.cu"]
+           "attn_merge.cu", "host_static.cu"]
 HEADERS = ["sm100.cuh", "wan_kernels.h"]
 LIB = os.path.join(PKG, "_lib", "libwanattn.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -11,7 +11,7 @@
 
 namespace {
 
-constexpr int32_t kAbiVersion = 9;
+constexpr int32_t kAbiVersion = 10;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -189,6 +189,8 @@ const char* wan_status_string(int32_t status) {
     case WAN_ERR_ALIAS: return "out overlaps qkv";
     case WAN_ERR_MEMORY_KIND:
       return "a host buffer is not page-locked, or a device buffer is not memory of the current device";
+    case WAN_ERR_TOO_LARGE:
+      return "the step does not fit wan_dit_attn_host_static's device buffer (WAN_HOST_STATIC_MAX_ELEMENTS)";
     case WAN_ERR_KERNEL_IMAGE:
       return "a compiled attention kernel's register count differs from the one its register split was "
              "written for: rebuild the library with the CUDA toolkit it targets";
@@ -511,6 +513,59 @@ int32_t wan_dit_attn_host(const void* qkv_host, void* out_host, void* qkv_dev, v
   WAN_TRY(check_device());
   WAN_TRY(check_memory_kind(qkv_host, out_host, qkv_dev, out_dev));
   (void)cudaGetLastError();
+  wan::HostStep step;
+  step.qkv_host = qkv_host;
+  step.out_host = out_host;
+  step.qkv_dev = qkv_dev;
+  step.out_dev = out_dev;
+  step.batch = batch;
+  step.S = S;
+  step.F = F;
+  step.H = H;
+  step.W = W;
+  step.heads = heads;
+  step.heads_per_chunk = hc;
+  step.gamma_q = gamma_q;
+  step.gamma_k = gamma_k;
+  step.eps = eps;
+  step.theta = theta;
+  step.scale = scale;
+  step.overlap_input = (flags & WAN_HOST_OVERLAP_INPUT) != 0;
+  WAN_LAUNCH_TRY(wan::enqueue_dit_attn_host(step, static_cast<cudaStream_t>(stream)));
+  return WAN_OK;
+}
+
+int32_t wan_dit_attn_host_static(const void* qkv_host, void* out_host, int64_t batch, int32_t F, int32_t H,
+                                 int32_t W, int32_t heads, int32_t head_dim, const void* gamma_q,
+                                 const void* gamma_k, float eps, float theta, float scale,
+                                 int32_t heads_per_chunk, int32_t flags, void* stream) {
+  int64_t S = 0;
+  WAN_TRY(check_heads(heads, head_dim));
+  WAN_TRY(check_grid(batch, F, H, W, heads, &S));
+  if (!qkv_host || !out_host || !gamma_q || !gamma_k) return WAN_ERR_NULL;
+  if (!aligned16(gamma_q) || !aligned16(gamma_k)) return WAN_ERR_ALIGN;
+  if (!(std::isfinite(eps) && eps > 0.f) || !(std::isfinite(theta) && theta > 1.f)) return WAN_ERR_PARAM;
+  if (!std::isfinite(scale)) return WAN_ERR_PARAM;
+  if (heads_per_chunk < 0 || heads_per_chunk > heads) return WAN_ERR_PARAM;
+  if (flags & ~WAN_HOST_OVERLAP_INPUT) return WAN_ERR_PARAM;
+  const int32_t hc = heads_per_chunk > 0 ? heads_per_chunk
+                                         : (heads < WAN_HOST_HEADS_PER_CHUNK ? heads : WAN_HOST_HEADS_PER_CHUNK);
+  if (batch * ((heads + hc - 1) / hc) > WAN_HOST_MAX_PIECES) return WAN_ERR_SHAPE;
+  // batch * S * heads * 128 elements must fit the library's static buffer.
+  if (batch > WAN_HOST_STATIC_MAX_ELEMENTS / (S * heads * WAN_HEAD_DIM)) return WAN_ERR_TOO_LARGE;
+  WAN_TRY(check_device());
+  for (const void* p : {qkv_host, static_cast<const void*>(out_host)}) {
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return WAN_ERR_MEMORY_KIND;
+    }
+    if (at.type != cudaMemoryTypeHost) return WAN_ERR_MEMORY_KIND;
+  }
+  (void)cudaGetLastError();
+  void* qkv_dev = nullptr;
+  void* out_dev = nullptr;
+  if (wan::host_static_buffers(&qkv_dev, &out_dev) != cudaSuccess) return WAN_ERR_LAUNCH;
   wan::HostStep step;
   step.qkv_host = qkv_host;
   step.out_host = out_host;

@@ -114,6 +114,12 @@ struct HostStep {
 };
 cudaError_t enqueue_dit_attn_host(const HostStep& step, cudaStream_t stream);
 
+// The library's own staging buffers for the host-buffer step (host_static.cu):
+// packed QKV and output regions of one static device array, at fixed
+// offsets, on the current device. The first call on a device looks the
+// array's address up.
+cudaError_t host_static_buffers(void** qkv_dev, void** out_dev);
+
 // FP8 (e4m3) variant (fp8_quant.cu, attn_fwd_fp8.cu). Codes of X are
 // e4m3(fl32(x * inv_X)); the attention dequantises with scale_X. qk8 is
 // [B][S][2D] (Q then K codes of each token), v8t [B][heads][128][s_pitch]

@@ -47,6 +47,7 @@ cudaError_t launch_qk_norm_rope(void* qkv, int64_t batch, int32_t F, int32_t H, 
 struct AttnPlan {
   alignas(64) unsigned char tmap[128];     // CUtensorMap over the buffer holding Q
   alignas(64) unsigned char tmap_kv[128];  // CUtensorMap over the buffer holding K and V
+  const void* q_base;                      // the buffer holding Q ([batch][S][3D])
   void* out;
   int32_t S, heads, D, q_pairs, n_kv;
   float scale_log2;

@@ -267,3 +267,22 @@ def test_header_compiles_as_c_and_links(lib, tmp_path):
     assert all(texts) and len(set(texts)) == 13
     assert out[14] == "null 1"          # WAN_ERR_NULL
     assert out[15] == "head_dim 4"      # WAN_ERR_HEAD_DIM
+
+
+def test_build_refuses_a_split_register_kernel_with_another_register_count():
+    """The per-warpgroup register split is only valid at the register count
+    the source names: a ptxas report with another count fails the build."""
+    name = "_ZN3wan44_GLOBAL__N__fa96f1d5_11_attn_fwd_cu_a33b3c8a15attn_fwd_kernelILb0ELb0EEEv14CUtensorMap_st"
+    fp8 = "_ZN3wan45_GLOBAL__N__2abe_12_attn_fwd_fp8_cu_2abe942719attn_fwd_fp8_kernelE14CUtensorMap_st"
+    import re as _re
+    want = {src: int(_re.search(r"constexpr int kLaunchRegs = (\d+);", open(os.path.join(wan_build.CSRC, src)).read()).group(1))
+            for src, _ in wan_build.SPLIT_REGISTER_KERNELS
+            if _re.search(r"constexpr int kLaunchRegs", open(os.path.join(wan_build.CSRC, src)).read())}
+    good = (f"ptxas info    : Compiling entry function '{name}' for 'sm_100a'\n"
+            f"ptxas info    : Used {want.get('attn_fwd.cu', 168)} registers, used 1 barriers\n"
+            f"ptxas info    : Compiling entry function '{fp8}' for 'sm_100a'\n"
+            f"ptxas info    : Used {want.get('attn_fwd_fp8.cu', 168)} registers, used 1 barriers\n")
+    wan_build.check_register_splits(good)
+    bad = good.replace(f"Used {want.get('attn_fwd_fp8.cu', 168)} registers", "Used 170 registers")
+    with pytest.raises(RuntimeError, match="kLaunchRegs"):
+        wan_build.check_register_splits(bad)

@@ -9,6 +9,7 @@ from __future__ import annotations
 
 import argparse
 import os
+import re
 import shutil
 import subprocess
 import sys
@@ -44,6 +45,33 @@ def stale() -> bool:
     return any(os.path.getmtime(f) > t for f in _inputs())
 
 
+# Kernels that split their registers between warpgroups with setmaxnreg: the
+# split is only valid when the compiled kernel launches with exactly the
+# register count its source names (kLaunchRegs). (source file, kernel name)
+SPLIT_REGISTER_KERNELS = [("attn_fwd.cu", "attn_fwd_kernel"), ("attn_fwd_fp8.cu", "attn_fwd_fp8_kernel")]
+
+
+def check_register_splits(ptxas_log: str) -> None:
+    """Fail the build when a split-register kernel did not compile to the
+    register count its source assumes (ptxas -v: 'Used N registers' after
+    'Compiling entry function <name>')."""
+    entries = re.findall(r"Compiling entry function '([^']+)'.*?Used (\d+) registers", ptxas_log, re.S)
+    for src, kernel in SPLIT_REGISTER_KERNELS:
+        text = open(os.path.join(CSRC, src)).read()
+        m = re.search(r"constexpr int kLaunchRegs = (\d+);", text)
+        if m is None:
+            continue  # this kernel no longer splits its registers
+        want = int(m.group(1))
+        found = [(name, int(n)) for name, n in entries if kernel in name and src.replace(".", "_") in name]
+        if not found:
+            raise RuntimeError(f"ptxas reported no entry function {kernel} of {src}")
+        bad = [(name, n) for name, n in found if n != want]
+        if bad:
+            raise RuntimeError(f"{kernel} ({src}) compiled to {bad[0][1]} registers per thread; its per-warpgroup "
+                               f"register split (setmaxnreg) assumes kLaunchRegs = {want}. Adjust kLaunchRegs and "
+                               f"the split, or build with the toolkit the source was tuned for.")
+
+
 def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
     if not force and not stale():
         return LIB
@@ -51,11 +79,18 @@ def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
     tmp = LIB + f".{os.getpid()}.tmp"
     cmd = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
            "-Xcompiler", "-fvisibility=hidden", "--expt-relaxed-constexpr",
-           "-I", os.path.join(ROOT, "include"), *extra_flags]
-    if verbose:
-        cmd += ["-Xptxas", "-v"]
+           "-I", os.path.join(ROOT, "include"), "-Xptxas", "-v", *extra_flags]
     cmd += [os.path.join(CSRC, f) for f in SOURCES] + ["-o", tmp]
-    subprocess.check_call(cmd)
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    if verbose or res.returncode != 0:
+        sys.stderr.write(res.stdout + res.stderr)
+    if res.returncode != 0:
+        raise subprocess.CalledProcessError(res.returncode, cmd, res.stdout, res.stderr)
+    try:
+        check_register_splits(res.stdout + res.stderr)
+    except RuntimeError:
+        os.remove(tmp)
+        raise
     os.replace(tmp, LIB)
     return LIB
 

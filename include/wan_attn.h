@@ -261,6 +261,12 @@ WAN_API int32_t wan_self_attention_rows(const void* qkv, void* out, int64_t batc
  *   O uses the probabilities rounded to bf16, as (2) does, and so does l.
  *   All pointers 16-byte aligned; o and ml overlap neither input nor each
  *   other. The full row's output is merge(all ranges) finalised below.
+ * wan_self_attention_accumulate: as wan_self_attention_partial, but o and ml
+ *   already hold a state (over other keys, e.g. earlier ring rounds), and the
+ *   launch merges its own state into them (the merge below, done in the
+ *   attention's epilogue) instead of overwriting them: one launch per ring
+ *   round after the first, with no separate merge and no buffer for the
+ *   round's own state.
  * wan_attention_merge: for n_units (row, head) units in the layouts above
  *   (n_units = batch * rows * heads): when o_part is not NULL,
  *   (o_acc, ml_acc) := the merge of itself and (o_part, ml_part):
@@ -275,6 +281,10 @@ WAN_API int32_t wan_self_attention_partial(const void* q_qkv, int64_t q_seq_len,
                                            const void* kv, int64_t kv_rows, int64_t kv_pitch, int64_t k_row0,
                                            int64_t k_rows, float* o, float* ml, int64_t batch, int32_t heads,
                                            int32_t head_dim, float scale, void* stream);
+WAN_API int32_t wan_self_attention_accumulate(const void* q_qkv, int64_t q_seq_len, int64_t q_row0,
+                                              int64_t q_rows, const void* kv, int64_t kv_rows, int64_t kv_pitch,
+                                              int64_t k_row0, int64_t k_rows, float* o, float* ml, int64_t batch,
+                                              int32_t heads, int32_t head_dim, float scale, void* stream);
 WAN_API int32_t wan_attention_merge(float* o_acc, float* ml_acc, const float* o_part, const float* ml_part,
                                     void* out, int64_t n_units, int32_t head_dim, void* stream);
 

@@ -39,7 +39,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings(lib):
-    assert lib.wan_abi_version() == 10
+    assert lib.wan_abi_version() == 11
     for code in range(13):
         assert lib.wan_status_string(code)
     assert lib.wan_status_string(99) == b"unknown status"
@@ -204,6 +204,11 @@ def test_ring_entry_points_validate(lib):
     assert call(sc=float("inf")) == 5
     assert call(o=FAKE + 16) == 9             # o overlaps q
     assert call(ml=far2 + 64) == 9            # ml overlaps o
+    # the accumulating form validates like the partial one
+    acc_args = list(ok)
+    assert lib.wan_self_attention_accumulate(*acc_args[:9], None, *acc_args[10:]) == 1
+    acc_args[13] = 64
+    assert lib.wan_self_attention_accumulate(*acc_args) == 4
     # wan_attention_merge(o_acc, ml_acc, o_part, ml_part, out, n_units, head_dim)
     assert lib.wan_attention_merge(far1, far2, None, None, None, 4, 128, None) == 1  # nothing to do
     assert lib.wan_attention_merge(far1, far2, far3, None, None, 4, 128, None) == 1  # o_part without ml_part

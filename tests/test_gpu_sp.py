@@ -211,3 +211,71 @@ def test_ring_and_gather_forms_on_a_side_stream():
                     dtype=np.int64)
     normed = oracle.qk_norm_rope(qkv, w.grid, w.heads, gq.cpu(), gk.cpu(), wi.EPS, wi.THETA)
     assert_attention_close(_sampled(w, out_r, rows), oracle.attention_rows(normed, w.heads, rows, SCALE), "ring")
+
+
+def test_ring_rounds_at_the_bench_shape_sampled_rows():
+    """The bench's ring side measurement, in its launch configuration: 8
+    simulated ranks over the 832x480, 81-frame CFG batch (2 x 32760 tokens,
+    40 heads), each rank's rounds over the 8 K|V chunks, partial states merged
+    round by round. Sampled rows of every rank (its first and last rows and
+    random ones) on the first and last heads of both batch elements, against
+    the oracle at the attention bound."""
+    w, d = _normed(2, seed=29)
+    world, D = 8, w.dim
+    s_local = w.seq_len // world
+    shards = [d[:, r * s_local:(r + 1) * s_local].contiguous() for r in range(world)]
+    chunks = [sh[..., D:].contiguous() for sh in shards]
+    acc = (torch.empty((w.batch, s_local, w.heads, 128), dtype=torch.float32, device="cuda"),
+           torch.empty((w.batch, s_local, w.heads, 2), dtype=torch.float32, device="cuda"))
+    part = (torch.empty_like(acc[0]), torch.empty_like(acc[1]))
+    outs = []
+    for r in range(world):
+        for i, c in enumerate(sp.ring_order(world, r)):
+            dst = acc if i == 0 else part
+            wan.self_attention_partial(shards[r], w.heads, chunks[c], o=dst[0], ml=dst[1])
+            if i > 0:
+                wan.attention_merge(acc[0], acc[1], part[0], part[1])
+        outs.append(wan.attention_merge(acc[0], acc[1], finalize=True))
+    torch.cuda.synchronize()
+    assert wan.device_error() == 0
+    out = torch.cat(outs, dim=1)
+    local = wi.sample_rows(s_local, 3, seed=30).numpy()
+    idx_rows = np.concatenate([r * s_local + local for r in range(world)])
+    rows = np.array([(b, h, i) for b in range(w.batch) for h in (0, w.heads - 1) for i in idx_rows], dtype=np.int64)
+    ref = oracle.attention_rows(d.cpu(), w.heads, rows, SCALE)
+    assert_attention_close(_sampled(w, out, rows), ref, "ring at the bench shape")
+
+
+@pytest.mark.parametrize("idx,world", [(1, 4), (4, 2)])
+def test_ring_rounds_accumulated_in_the_epilogue(idx, world):
+    """The ring rounds with every round after the first merged into the
+    running state by the attention's epilogue (wan_self_attention_accumulate),
+    against the oracle on sampled rows of every rank, and against the same
+    rounds merged by the separate merge kernel (same arithmetic, so the two
+    agree to fp32 rounding)."""
+    w, d = _normed(idx, seed=31 + world)
+    S, D = w.seq_len, w.dim
+    s_local = S // world
+    shards = [d[:, r * s_local:(r + 1) * s_local].contiguous() for r in range(world)]
+    chunks = [sh[..., D:].contiguous() for sh in shards]
+    outs_acc, outs_merge = [], []
+    for r in range(world):
+        order = sp.ring_order(world, r)
+        o, ml = wan.self_attention_partial(shards[r], w.heads, chunks[order[0]])
+        o2, ml2 = o.clone(), ml.clone()
+        for c in order[1:]:
+            wan.self_attention_partial(shards[r], w.heads, chunks[c], o=o, ml=ml, accumulate=True)
+            part = wan.self_attention_partial(shards[r], w.heads, chunks[c])
+            wan.attention_merge(o2, ml2, part[0], part[1])
+        outs_acc.append(wan.attention_merge(o, ml, finalize=True))
+        outs_merge.append(wan.attention_merge(o2, ml2, finalize=True))
+    torch.cuda.synchronize()
+    assert wan.device_error() == 0
+    out = torch.cat(outs_acc, dim=1)
+    assert float((out.float() - torch.cat(outs_merge, dim=1).float()).abs().max()) <= 1e-2
+    local = wi.sample_rows(s_local, 6, seed=32).numpy()
+    idx_rows = np.concatenate([r * s_local + local for r in range(world)])
+    rows = np.array([(b, h, i) for b in range(w.batch) for h in (0, w.heads - 1) for i in idx_rows],
+                    dtype=np.int64)
+    ref = oracle.attention_rows(d.cpu(), w.heads, rows, SCALE)
+    assert_attention_close(_sampled(w, out, rows), ref, f"accumulated ring world {world}")

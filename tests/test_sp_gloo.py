@@ -114,16 +114,17 @@ def _oracle_ring_ops(full_in, gq, gk, seen):
             r.wait()
         return buf
 
-    def attend(qkv_local, kv):
+    def attend(qkv_local, kv, state):
         B, s_local, _ = qkv_local.shape
         seen.append(kv[0, 0, 0].item())  # which chunk this round met (its first K value)
         rows = [(b, h, i) for b in range(B) for i in range(s_local) for h in range(HEADS)]
-        return oracle.attention_partial_rows(qkv_local, HEADS, kv, 0, kv.shape[1], rows, scale)
+        part = oracle.attention_partial_rows(qkv_local, HEADS, kv, 0, kv.shape[1], rows, scale)
+        return part if state is None else oracle.merge_partial(state, part)
 
     def finalize(state):
         return torch.from_numpy(oracle.finalize_partial(state)).view(BATCH, -1, HEADS * 128)
 
-    return sp.RingOps(norm_shard, kv_chunk, exchange, received, attend, oracle.merge_partial, finalize)
+    return sp.RingOps(norm_shard, kv_chunk, exchange, received, attend, finalize)
 
 
 def _ring_worker(rank, world, port, results):

@@ -98,6 +98,8 @@ def load_library() -> ctypes.CDLL:
             lib.wan_self_attention_partial.argtypes = [P, I64, I64, I64, P, I64, I64, I64, I64, P, P, I64, I32,
                                                        I32, F, P]
             lib.wan_self_attention_partial.restype = I32
+            lib.wan_self_attention_accumulate.argtypes = lib.wan_self_attention_partial.argtypes
+            lib.wan_self_attention_accumulate.restype = I32
             lib.wan_attention_merge.argtypes = [P, P, P, P, P, I64, I32, P]
             lib.wan_attention_merge.restype = I32
             lib.wan_dit_attn_host_static.argtypes = [P, P, I64, I32, I32, I32, I32, I32, P, P, F, F, F, I32, I32, P]
@@ -343,12 +345,14 @@ def _f32_cuda(t, name: str) -> int:
 
 
 def self_attention_partial(q_qkv, heads: int, kv, q_row0: int = 0, q_rows=None, k_row0: int = 0, k_rows=None,
-                           o=None, ml=None, scale: float = 0.0, stream=None):
+                           o=None, ml=None, scale: float = 0.0, stream=None, accumulate: bool = False):
     """Softmax state of query rows [q_row0, q_row0 + q_rows) of the packed
     q_qkv [B, Sq, 3*heads*128] against keys [k_row0, k_row0 + k_rows) of kv
     [B, Skv, pitch] (K then V in its last 2*heads*128 columns: a packed QKV
     buffer or a K|V chunk). Returns (o [B, q_rows, heads, 128] fp32,
-    ml [B, q_rows, heads, 2] fp32): O and (m, l) in base 2."""
+    ml [B, q_rows, heads, 2] fp32): O and (m, l) in base 2. With accumulate,
+    o and ml must hold a state over other keys already, and the range's state
+    is merged into them (wan_self_attention_accumulate)."""
     import torch
     _check_packed(q_qkv, heads)
     B, Sq, _ = q_qkv.shape
@@ -362,10 +366,12 @@ def self_attention_partial(q_qkv, heads: int, kv, q_row0: int = 0, q_rows=None, 
         ml = torch.empty((B, q_rows, heads, 2), dtype=torch.float32, device=q_qkv.device)
     if tuple(o.shape) != (B, q_rows, heads, HEAD_DIM) or tuple(ml.shape) != (B, q_rows, heads, 2):
         raise ValueError("o must be [B, q_rows, heads, 128] and ml [B, q_rows, heads, 2]")
-    _check(load_library().wan_self_attention_partial(
-        _bf16_cuda(q_qkv, "q_qkv"), Sq, int(q_row0), int(q_rows), _bf16_cuda(kv, "kv"), kv.shape[1], kv.shape[2],
-        int(k_row0), int(k_rows), _f32_cuda(o, "o"), _f32_cuda(ml, "ml"), B, heads, HEAD_DIM, scale,
-        _stream(stream)), "wan_self_attention_partial")
+    if accumulate and (o is None or ml is None):
+        raise ValueError("accumulate needs the state (o, ml) to merge into")
+    fn = load_library().wan_self_attention_accumulate if accumulate else load_library().wan_self_attention_partial
+    _check(fn(_bf16_cuda(q_qkv, "q_qkv"), Sq, int(q_row0), int(q_rows), _bf16_cuda(kv, "kv"), kv.shape[1],
+              kv.shape[2], int(k_row0), int(k_rows), _f32_cuda(o, "o"), _f32_cuda(ml, "ml"), B, heads, HEAD_DIM,
+              scale, _stream(stream)), "wan_self_attention_accumulate" if accumulate else "wan_self_attention_partial")
     return o, ml
 
 

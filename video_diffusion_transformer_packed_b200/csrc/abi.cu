@@ -11,7 +11,7 @@
 
 namespace {
 
-constexpr int32_t kAbiVersion = 10;
+constexpr int32_t kAbiVersion = 11;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -398,10 +398,13 @@ int32_t wan_self_attention_rows(const void* qkv, void* out, int64_t batch, int64
   return WAN_OK;
 }
 
-int32_t wan_self_attention_partial(const void* q_qkv, int64_t q_seq_len, int64_t q_row0, int64_t q_rows,
-                                   const void* kv, int64_t kv_rows, int64_t kv_pitch, int64_t k_row0,
-                                   int64_t k_rows, float* o, float* ml, int64_t batch, int32_t heads,
-                                   int32_t head_dim, float scale, void* stream) {
+}  // extern "C"
+
+namespace {
+int32_t partial_attention(const void* q_qkv, int64_t q_seq_len, int64_t q_row0, int64_t q_rows, const void* kv,
+                          int64_t kv_rows, int64_t kv_pitch, int64_t k_row0, int64_t k_rows, float* o, float* ml,
+                          int64_t batch, int32_t heads, int32_t head_dim, float scale, bool accumulate,
+                          void* stream) {
   WAN_TRY(check_heads(heads, head_dim));
   WAN_TRY(check_tokens(batch, q_seq_len, heads));
   if (!q_qkv || !kv || !o || !ml) return WAN_ERR_NULL;
@@ -434,8 +437,28 @@ int32_t wan_self_attention_partial(const void* q_qkv, int64_t q_seq_len, int64_t
   plan.q_rows = static_cast<int32_t>(q_rows);
   plan.o_part = o;
   plan.ml_part = ml;
+  plan.accumulate = accumulate;
   WAN_LAUNCH_TRY(wan::launch_attn_fwd(plan, static_cast<cudaStream_t>(stream), false));
   return WAN_OK;
+}
+}  // namespace
+
+extern "C" {
+
+int32_t wan_self_attention_partial(const void* q_qkv, int64_t q_seq_len, int64_t q_row0, int64_t q_rows,
+                                   const void* kv, int64_t kv_rows, int64_t kv_pitch, int64_t k_row0,
+                                   int64_t k_rows, float* o, float* ml, int64_t batch, int32_t heads,
+                                   int32_t head_dim, float scale, void* stream) {
+  return partial_attention(q_qkv, q_seq_len, q_row0, q_rows, kv, kv_rows, kv_pitch, k_row0, k_rows, o, ml, batch,
+                           heads, head_dim, scale, false, stream);
+}
+
+int32_t wan_self_attention_accumulate(const void* q_qkv, int64_t q_seq_len, int64_t q_row0, int64_t q_rows,
+                                      const void* kv, int64_t kv_rows, int64_t kv_pitch, int64_t k_row0,
+                                      int64_t k_rows, float* o, float* ml, int64_t batch, int32_t heads,
+                                      int32_t head_dim, float scale, void* stream) {
+  return partial_attention(q_qkv, q_seq_len, q_row0, q_rows, kv, kv_rows, kv_pitch, k_row0, k_rows, o, ml, batch,
+                           heads, head_dim, scale, true, stream);
 }
 
 int32_t wan_attention_merge(float* o_acc, float* ml_acc, const float* o_part, const float* ml_part, void* out,

@@ -93,6 +93,7 @@ struct AttnParams {
   uint16_t* out;
   float* o_part;   // partial mode (not null): fp32 unnormalised O instead of out
   float* ml_part;  // partial mode: (m, l) of every (row, head)
+  int32_t accumulate;  // partial mode: merge into (o_part, ml_part) instead of overwriting them
   int32_t k_rows;  // keys [k_row0, k_row0 + k_rows) of the K/V map
   int32_t k_row0;
   int32_t kv_k0, kv_v0;  // columns of K and V of head 0 in the K/V map
@@ -465,8 +466,19 @@ __device__ void run_softmax(const AttnParams& p, Bars bars, volatile int* abort,
   const int row = (2 * qp + t) * kBM + quarter * 32 + lane;  // within this launch's query rows
   const int64_t unit = (static_cast<int64_t>(b) * p.q_rows + row) * p.heads + h;
   if constexpr (kPartial) {
-    // Partial mode: the unnormalised state of this key range, for a merge.
+    // Partial mode: the unnormalised state of this key range, for a merge;
+    // with `accumulate`, merged here into the state already in (o_part,
+    // ml_part): both sides rescaled to the larger reference max.
     float4* dst = reinterpret_cast<float4*>(p.o_part + unit * kHD);
+    float w_new = 1.f, w_old = 0.f;
+    float2 ml = make_float2(m_run, l_run);
+    if (p.accumulate && row < p.q_rows) {
+      const float2 acc = reinterpret_cast<const float2*>(p.ml_part)[unit];
+      const float m = fmaxf(acc.x, m_run);
+      w_old = exp2f(acc.x - m);
+      w_new = exp2f(m_run - m);
+      ml = make_float2(m, acc.y * w_old + l_run * w_new);
+    }
 #pragma unroll 1
     for (int c = 0; c < 4; ++c) {
       uint32_t o[32];
@@ -475,12 +487,18 @@ __device__ void run_softmax(const AttnParams& p, Bars bars, volatile int* abort,
       if (row < p.q_rows) {
 #pragma unroll
         for (int v = 0; v < 8; ++v) {
-          dst[8 * c + v] = make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
-                                       __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3]));
+          float4 r = make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
+                                 __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3]));
+          if (p.accumulate) {
+            const float4 a = dst[8 * c + v];
+            r = make_float4(a.x * w_old + r.x * w_new, a.y * w_old + r.y * w_new, a.z * w_old + r.z * w_new,
+                            a.w * w_old + r.w * w_new);
+          }
+          dst[8 * c + v] = r;
         }
       }
     }
-    if (row < p.q_rows) reinterpret_cast<float2*>(p.ml_part)[unit] = make_float2(m_run, l_run);
+    if (row < p.q_rows) reinterpret_cast<float2*>(p.ml_part)[unit] = ml;
     return;
   } else {
   const float inv_l = 1.f / l_run;
@@ -664,6 +682,7 @@ cudaError_t plan_attn_fwd(const void* qkv, void* out, int64_t batch, int64_t seq
   plan->kv_v0 = 2 * D;
   plan->o_part = nullptr;
   plan->ml_part = nullptr;
+  plan->accumulate = false;
   return cudaSuccess;
 }
 
@@ -690,6 +709,7 @@ cudaError_t launch_attn_fwd(const AttnPlan& plan, cudaStream_t stream, bool pdl,
   p.out = static_cast<uint16_t*>(plan.out);
   p.o_part = plan.o_part;
   p.ml_part = plan.ml_part;
+  p.accumulate = plan.accumulate ? 1 : 0;
   p.k_rows = plan.k_rows;
   p.k_row0 = plan.k_row0;
   p.kv_k0 = plan.kv_k0;
@@ -717,7 +737,8 @@ cudaError_t launch_attn_fwd(const AttnPlan& plan, cudaStream_t stream, bool pdl,
       plan.q_row0 < 0 || plan.q_rows < 1 || static_cast<int64_t>(plan.q_row0) + plan.q_rows > plan.S ||
       plan.k_row0 < 0 || plan.k_rows < 1 || plan.n_kv != (plan.k_rows + kBN - 1) / kBN ||
       (plan.o_part != nullptr) != (plan.ml_part != nullptr) ||
-      (plan.o_part != nullptr && plan.skip_threshold > 0.f) || grid > INT32_MAX) {
+      (plan.o_part != nullptr && plan.skip_threshold > 0.f) || (plan.accumulate && plan.o_part == nullptr) ||
+      grid > INT32_MAX) {
     return cudaErrorInvalidValue;
   }
   cfg.gridDim = dim3(static_cast<unsigned>(grid));

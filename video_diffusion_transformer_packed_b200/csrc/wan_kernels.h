@@ -70,6 +70,10 @@ struct AttnPlan {
   // l = sum_j 2^(a_j - m) over the key range, a_j = scale log2(e) q . k_j.
   float* o_part;
   float* ml_part;
+  // Partial mode with accumulate: (o_part, ml_part) already hold a state over
+  // other keys, and the launch merges its own into it (each side rescaled to
+  // the larger m) instead of overwriting it.
+  bool accumulate;
 };
 
 cudaError_t plan_attn_fwd(const void* qkv, void* out, int64_t batch, int64_t seq_len,

@@ -15,9 +15,11 @@ All-gather form (`sequence_parallel_step`), the page's fallback:
 Ring form (`ring_attention_step`), the page's ring attention: after step 1,
 the K|V columns of the shard travel around the ring, one neighbour exchange
 per round, and each round's attention of the local queries against the chunk
-in hand runs while the next chunk is in flight. A round yields the softmax
-state of its key range (wan_self_attention_partial); the states merge exactly
-(wan_attention_merge), and no rank ever holds the full K/V. A chunk is 2/3 of
+in hand runs while the next chunk is in flight. A round folds the softmax
+state of its key range into the rank's running state (the first round
+writes it, wan_self_attention_partial; later rounds merge in the attention's
+epilogue, wan_self_attention_accumulate), and the final state is normalised
+(wan_attention_merge). No rank ever holds the full K/V. A chunk is 2/3 of
 the bytes the all-gather moves per token (no Q).
 
 Compute is only ever the CUDA kernels of this package (`cuda_ops`,
@@ -119,9 +121,10 @@ class RingOps:
     exchange(kv) -> handle             start sending kv to rank + 1 and
                                        receiving the next chunk from rank - 1
     received(handle) -> kv             the received chunk, once it is in
-    attend(qkv_local, kv) -> state     softmax state of the local queries
-                                       against the keys of kv
-    merge(state, part) -> state        fold a round's state in
+    attend(qkv_local, kv, state) -> state
+                                       the softmax state of the local queries
+                                       against the keys of kv, folded into
+                                       `state` (None in the first round)
     finalize(state) -> out             [B, s_local, heads*128]
     """
     norm_shard: Callable
@@ -129,7 +132,6 @@ class RingOps:
     exchange: Callable
     received: Callable
     attend: Callable
-    merge: Callable
     finalize: Callable
 
 
@@ -141,7 +143,7 @@ def ring_order(world: int, rank: int):
 
 def ring_attention_step(qkv_local, grid: Sequence[int], world: int, rank: int, ops: RingOps):
     """One rank's share in ring form: norm its shard in place, then `world`
-    rounds of (start the next exchange, attend the chunk in hand, merge)."""
+    rounds of (start the next exchange, fold the chunk in hand into the state)."""
     F, H, W = grid
     s0, s_local = shard_bounds(F * H * W, world, rank)
     if qkv_local.shape[1] != s_local:
@@ -151,16 +153,16 @@ def ring_attention_step(qkv_local, grid: Sequence[int], world: int, rank: int, o
     state = None
     for i in range(world):
         handle = ops.exchange(kv) if i + 1 < world else None  # in flight during this round's attention
-        part = ops.attend(qkv_local, kv)
-        state = part if state is None else ops.merge(state, part)
+        state = ops.attend(qkv_local, kv, state)
         if handle is not None:
             kv = ops.received(handle)
     return ops.finalize(state)
 
 
 def cuda_ring_ops(grid: Sequence[int], heads: int, gamma_q, gamma_k, group=None, stream=None) -> RingOps:
-    """The package's kernels in ring form: the partial-state attention and the
-    merge on `stream` (default: the current stream), K|V chunks exchanged with
+    """The package's kernels in ring form: the round's attention merged into
+    the running state in its epilogue, on `stream` (default: the current
+    stream), K|V chunks exchanged with
     the ring neighbours by NCCL point-to-point messages. The messages are
     enqueued before the round's attention and are ordered after the work
     already on the stream (the chunk being sent is complete); the next round's
@@ -203,17 +205,14 @@ def cuda_ring_ops(grid: Sequence[int], heads: int, gamma_q, gamma_k, group=None,
                 r.wait()
         return buf
 
-    def attend(qkv_local, kv):
+    def attend(qkv_local, kv, state):
         with _on_stream(stream):
-            return wan.self_attention_partial(qkv_local, heads, kv)
-
-    def merge(state, part):
-        with _on_stream(stream):
-            wan.attention_merge(state[0], state[1], part[0], part[1])
-        return state
+            if state is None:
+                return wan.self_attention_partial(qkv_local, heads, kv)
+            return wan.self_attention_partial(qkv_local, heads, kv, o=state[0], ml=state[1], accumulate=True)
 
     def finalize(state):
         with _on_stream(stream):
             return wan.attention_merge(state[0], state[1], finalize=True)
 
-    return RingOps(norm_shard, kv_chunk, exchange, received, attend, merge, finalize)
+    return RingOps(norm_shard, kv_chunk, exchange, received, attend, finalize)

@@ -16,7 +16,9 @@
 //   warp 9      MMA issuer (one thread): tcgen05.mma S_t = Q_t K_j^T into
 //               TMEM, then O_t += P_t V_j with P_t read from TMEM. The two
 //               query tiles ping-pong: while one tile's softmax runs, the
-//               tensor core works on the other tile.
+//               tensor core works on the other tile. The key loop is unrolled
+//               by four, so that ring slots and barrier parities are
+//               constants in the issuer's instruction stream.
 //   warps 0-3   softmax of tile 0, warps 4-7 softmax of tile 1: thread r owns
 //               query row r (TMEM lane r). Online softmax in base 2; the
 //               running max is only raised (and O rescaled in TMEM) when a
@@ -36,6 +38,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 
 #include "sm100.cuh"
 #include "wan_kernels.h"
@@ -69,7 +72,7 @@ constexpr uint32_t kAllGroupsSkipped = 0x01010101u;  // Skip-Softmax votes of th
 // P_t is handed to the MMA issuer in kPParts column blocks, each with its own
 // barrier: O_t += P_t V starts on the first keys while the softmax is still
 // exponentiating the last ones.
-constexpr int kPParts = 2;
+constexpr int kPParts = 4;
 constexpr int kPairsPerPart = 64 / kPParts;  // bf16 pairs (TMEM columns) per block
 static_assert(kPParts == 1 || kPParts == 2 || kPParts == 4, "P blocks");
 
@@ -242,16 +245,18 @@ __device__ void run_mma(const AttnParams& p, uint32_t smem, Bars bars, volatile 
     mma_commit(bars.s_full(1));
     mma_commit(bars.kv_empty(0));
   }
-#pragma unroll 1
-  for (int j = 0; j < p.n_kv && ok; ++j) {
-    const int iv = 2 * j + 1, ik = 2 * j + 2;
-    const int sv = iv % kStages, sk = ik % kStages;
+  auto step = [&](int j, auto rc) -> bool {
+    constexpr int r = decltype(rc)::value;  // j % 4
+    constexpr int sv = (2 * r + 1) % kStages, sk = (2 * r + 2) % kStages;
+    // phase parities of the ring slots for items 2j+1, 2j+2, 2j+3
+    constexpr uint32_t kpv = ((2 * r + 1) / kStages) & 1, kpk = ((2 * r + 2) / kStages) & 1,
+                       kpn = ((2 * r + 3) / kStages) & 1;
     const bool more = j + 1 < p.n_kv;
     const uint32_t acc = j > 0 ? 1u : 0u;
-    const uint32_t pj = j & 1;
-    if (!ensure(next_v, kv_bar(iv), kv_par(iv)) || !ensure(next_p, bars.p_full(0, 0), pj)) {
+    constexpr uint32_t pj = r & 1;
+    if (!ensure(next_v, bars.kv_full(sv), kpv) || !ensure(next_p, bars.p_full(0, 0), pj)) {
       ok = false;
-      break;
+      return false;
     }
     // O_0 += P_0 V_j, one block of P at a time.
     bool probe = false;
@@ -271,14 +276,14 @@ __device__ void run_mma(const AttnParams& p, uint32_t smem, Bars bars, volatile 
         const int k0 = part * kStepsPerPart, k1 = k0 + kStepsPerPart;
         pv_steps(0, sv, k0, k1 - 1, acc);
         probe = part + 1 < kPParts ? mbar_test(bars.p_full(0, part + 1), pj)
-                                   : (more ? mbar_test(kv_bar(ik), kv_par(ik)) : true);
+                                   : (more ? mbar_test(bars.kv_full(sk), kpk) : true);
         pv_steps(0, sv, k1 - 1, k1, acc);
       }
     }
-    if (!ok) break;
+    if (!ok) return false;
     if (more) {
       // S_0 = Q_0 K_{j+1}^T
-      if (!ensure(probe, kv_bar(ik), kv_par(ik))) { ok = false; break; }
+      if (!ensure(probe, bars.kv_full(sk), kpk)) { ok = false; return false; }
       qk_steps(0, sk, 0, 7);
       probe = mbar_test(bars.p_full(1, 0), pj);
       qk_steps(0, sk, 7, 8);
@@ -287,7 +292,7 @@ __device__ void run_mma(const AttnParams& p, uint32_t smem, Bars bars, volatile 
       probe = mbar_test(bars.p_full(1, 0), pj);
     }
     // O_1 += P_1 V_j
-    if (!ensure(probe, bars.p_full(1, 0), pj)) { ok = false; break; }
+    if (!ensure(probe, bars.p_full(1, 0), pj)) { ok = false; return false; }
     if (kSkip && votes[1] == kAllGroupsSkipped) {
 #pragma unroll
       for (int part = 1; part < kPParts; ++part) {
@@ -304,17 +309,32 @@ __device__ void run_mma(const AttnParams& p, uint32_t smem, Bars bars, volatile 
         pv_steps(1, sv, k1 - 1, k1, acc);
       }
     }
-    if (!ok) break;
+    if (!ok) return false;
     mma_commit(bars.kv_empty(sv));
     if (more) {
       // S_1 = Q_1 K_{j+1}^T; probe what the next iteration starts with.
       qk_steps(1, sk, 0, 7);
-      next_v = mbar_test(kv_bar(iv + 2), kv_par(iv + 2));
+      next_v = mbar_test(bars.kv_full((sv + 2) % kStages), kpn);
       next_p = mbar_test(bars.p_full(0, 0), pj ^ 1u);
       qk_steps(1, sk, 7, 8);
       mma_commit(bars.s_full(1));
       mma_commit(bars.kv_empty(sk));
     }
+    return true;
+  };
+  // Key tiles in fours: K_j and V_j take ring slots 2j % 4 and (2j+1) % 4,
+  // and a slot's phase parity repeats every four key tiles, so within a
+  // group every slot, descriptor offset and parity is a compile-time
+  // constant. The issuing thread is on the critical path (an MMA group starts
+  // only as fast as it forms the descriptors and barrier addresses), and this
+  // form issues the same MMAs with about a tenth fewer cycles per key tile.
+  static_assert(kStages == 4, "slot pattern");
+#pragma unroll 1
+  for (int j = 0; j < p.n_kv && ok; j += 4) {
+    ok = step(j, std::integral_constant<int, 0>{});
+    if (ok && j + 1 < p.n_kv) ok = step(j + 1, std::integral_constant<int, 1>{});
+    if (ok && j + 2 < p.n_kv) ok = step(j + 2, std::integral_constant<int, 2>{});
+    if (ok && j + 3 < p.n_kv) ok = step(j + 3, std::integral_constant<int, 3>{});
   }
   if (kSkip && n_pv_skipped) atomicAdd(&g_attn_skip_stats[1], n_pv_skipped);
   if (ok) {
@@ -571,7 +591,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_holder;
+  // Read through a shuffle, so that the compiler knows the TMEM base to be
+  // warp-uniform: the tcgen05 addresses derived from it are then formed in
+  // uniform registers instead of being moved there before every MMA.
+  const uint32_t tmem = __shfl_sync(0xffffffffu, *tmem_holder, 0);
 
   if (warp >= 8) {
     regs_decrease<kCtlRegs>();

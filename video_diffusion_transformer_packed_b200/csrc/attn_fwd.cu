@@ -69,12 +69,18 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait (the default limit)
 constexpr float kRescaleThreshold = 8.0f;         // log2 of the largest tolerated growth
 constexpr uint32_t kAllGroupsSkipped = 0x01010101u;  // Skip-Softmax votes of the four warps
-// P_t is handed to the MMA issuer in kPParts column blocks, each with its own
+// P_t is handed to the MMA issuer in column blocks, each with its own
 // barrier: O_t += P_t V starts on the first keys while the softmax is still
-// exponentiating the last ones.
+// exponentiating the last ones. kPParts barriers per tile are allocated; the
+// dense and partial kernels use four blocks, the Skip-Softmax kernel two (its
+// skipped tiles wait on every block, so more blocks cost it more than they
+// overlap).
 constexpr int kPParts = 4;
-constexpr int kPairsPerPart = 64 / kPParts;  // bf16 pairs (TMEM columns) per block
-static_assert(kPParts == 1 || kPParts == 2 || kPParts == 4, "P blocks");
+template <bool kSkip>
+constexpr int p_parts() { return kSkip ? 2 : 4; }
+static_assert(p_parts<false>() <= kPParts && p_parts<true>() <= kPParts, "P blocks");
+static_assert((64 / p_parts<false>()) % 16 == 0 && (64 / p_parts<true>()) % 16 == 0,
+              "P is stored in 16-column pieces");
 
 // Shared memory map (offsets from a 1024-byte aligned base).
 constexpr int kOffQ = 0;                              // 2 tiles
@@ -228,7 +234,8 @@ __device__ void run_mma(const AttnParams& p, uint32_t smem, Bars bars, volatile 
     tc_fence_after();
     return true;
   };
-  constexpr int kStepsPerPart = 8 / kPParts;
+  constexpr int kParts = p_parts<kSkip>();
+  constexpr int kStepsPerPart = 8 / kParts;
   auto kv_bar = [&](int i) { return bars.kv_full(i % kStages); };
   auto kv_par = [&](int i) { return static_cast<uint32_t>((i / kStages) & 1); };
 
@@ -265,17 +272,17 @@ __device__ void run_mma(const AttnParams& p, uint32_t smem, Bars bars, volatile 
       // blocks' arrivals are still awaited, so that the warps' stores of
       // P = 0 are done before S_0 is rewritten.
 #pragma unroll
-      for (int part = 1; part < kPParts; ++part) {
+      for (int part = 1; part < kParts; ++part) {
         if (!ensure(false, bars.p_full(0, part), pj)) { ok = false; break; }
       }
       ++n_pv_skipped;
     } else {
 #pragma unroll
-      for (int part = 0; part < kPParts; ++part) {
+      for (int part = 0; part < kParts; ++part) {
         if (part > 0 && !ensure(probe, bars.p_full(0, part), pj)) { ok = false; break; }
         const int k0 = part * kStepsPerPart, k1 = k0 + kStepsPerPart;
         pv_steps(0, sv, k0, k1 - 1, acc);
-        probe = part + 1 < kPParts ? mbar_test(bars.p_full(0, part + 1), pj)
+        probe = part + 1 < kParts ? mbar_test(bars.p_full(0, part + 1), pj)
                                    : (more ? mbar_test(bars.kv_full(sk), kpk) : true);
         pv_steps(0, sv, k1 - 1, k1, acc);
       }
@@ -295,17 +302,17 @@ __device__ void run_mma(const AttnParams& p, uint32_t smem, Bars bars, volatile 
     if (!ensure(probe, bars.p_full(1, 0), pj)) { ok = false; return false; }
     if (kSkip && votes[1] == kAllGroupsSkipped) {
 #pragma unroll
-      for (int part = 1; part < kPParts; ++part) {
+      for (int part = 1; part < kParts; ++part) {
         if (!ensure(false, bars.p_full(1, part), pj)) { ok = false; break; }
       }
       ++n_pv_skipped;
     } else {
 #pragma unroll
-      for (int part = 0; part < kPParts; ++part) {
+      for (int part = 0; part < kParts; ++part) {
         if (part > 0 && !ensure(probe, bars.p_full(1, part), pj)) { ok = false; break; }
         const int k0 = part * kStepsPerPart, k1 = k0 + kStepsPerPart;
         pv_steps(1, sv, k0, k1 - 1, acc);
-        probe = part + 1 < kPParts ? mbar_test(bars.p_full(1, part + 1), pj) : false;
+        probe = part + 1 < kParts ? mbar_test(bars.p_full(1, part + 1), pj) : false;
         pv_steps(1, sv, k1 - 1, k1, acc);
       }
     }
@@ -353,6 +360,8 @@ template <bool kSkip, bool kPartial>
 __device__ void run_softmax(const AttnParams& p, Bars bars, volatile int* abort, uint32_t tmem,
                             int t, int quarter, int lane, int b, int h, int qp,
                             volatile uint8_t* votes) {
+  constexpr int kParts = p_parts<kSkip>();
+  constexpr int kPairsPerPart = 64 / kParts;  // bf16 pairs (TMEM columns) per block
   const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
   const uint32_t tS = tmem + lane_base + t * 128;
   const uint32_t tO = tmem + lane_base + 256 + t * 128;
@@ -412,7 +421,7 @@ __device__ void run_softmax(const AttnParams& p, Bars bars, volatile int* abort,
         tmem_wait_st();
         tc_fence_before();
 #pragma unroll
-        for (int part = 0; part < kPParts; ++part) mbar_arrive(bars.p_full(t, part));
+        for (int part = 0; part < kParts; ++part) mbar_arrive(bars.p_full(t, part));
         ++n_skipped;
         continue;
       }
@@ -447,7 +456,7 @@ __device__ void run_softmax(const AttnParams& p, Bars bars, volatile int* abort,
     const uint64_t negm2 = f2(-m_run, -m_run);
     float sums[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // 8 chains
 #pragma unroll
-    for (int part = 0; part < kPParts; ++part) {
+    for (int part = 0; part < kParts; ++part) {
       uint32_t pk[kPairsPerPart];
 #pragma unroll
       for (int e = 0; e < kPairsPerPart; ++e) {
@@ -459,13 +468,9 @@ __device__ void run_softmax(const AttnParams& p, Bars bars, volatile int* abort,
         pk[e] = pack_bf16x2(p0, p1);
         add_bf16x2_f32(pk[e], sums[2 * (e & 3)], sums[2 * (e & 3) + 1]);
       }
-      if constexpr (kPairsPerPart == 64) {
-        tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(pk));
-        tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(pk + 32));
-      } else if constexpr (kPairsPerPart == 32) {
-        tmem_st32(tS + 32 * part, *reinterpret_cast<uint32_t(*)[32]>(pk));
-      } else {
-        tmem_st16(tS + 16 * part, *reinterpret_cast<uint32_t(*)[16]>(pk));
+#pragma unroll
+      for (int c = 0; c < kPairsPerPart / 16; ++c) {
+        tmem_st16(tS + kPairsPerPart * part + 16 * c, *reinterpret_cast<uint32_t(*)[16]>(pk + 16 * c));
       }
       tmem_wait_st();
       tc_fence_before();

@@ -16,6 +16,8 @@
 // code buffer [B][S][2D], V from the transposed buffer [B][heads][128][s_pitch],
 // so V^T tiles are K-major like the K tiles), warp 9 issues the MMAs, warps
 // 0-3 and 4-7 run the online softmax of the two query tiles in ping-pong.
+// The issuer's key loop is unrolled by eight, so that ring slots and barrier
+// parities are constants in its instruction stream.
 // An e4m3 tile of 128 x 128 is 16 KB, one 128-byte-swizzled box; a K = 32
 // step advances 32 bytes inside it. P_t (128 codes per row, four per 32-bit
 // column) is written over S_t in TMEM and handed over in two 64-key blocks.
@@ -31,6 +33,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 
 #include "sm100.cuh"
 #include "wan_kernels.h"
@@ -187,16 +190,18 @@ __device__ void run_mma(const AttnFp8Params& p, uint32_t smem, Bars bars, volati
     mma_commit(bars.s_full(1));
     mma_commit(bars.kv_empty(0));
   }
-#pragma unroll 1
-  for (int j = 0; j < p.n_kv && ok; ++j) {
-    const int iv = 2 * j + 1, ik = 2 * j + 2;
-    const int sv = iv % kStages, sk = ik % kStages;
+  auto step = [&](int j, auto rc) -> bool {
+    constexpr int r = decltype(rc)::value;  // j % 8
+    constexpr int sv = (2 * r + 1) % kStages, sk = (2 * r + 2) % kStages;
+    // phase parities of the ring slots of items 2j+1, 2j+2 and 2j+3
+    constexpr uint32_t kpv = ((2 * r + 1) / kStages) & 1, kpk = ((2 * r + 2) / kStages) & 1,
+                       kpn = ((2 * r + 3) / kStages) & 1;
     const bool more = j + 1 < p.n_kv;
     const uint32_t acc = j > 0 ? 1u : 0u;
-    const uint32_t pj = j & 1;
-    if (!ensure(next_v, kv_bar(iv), kv_par(iv)) || !ensure(next_p, bars.p_full(0, 0), pj)) {
+    constexpr uint32_t pj = r & 1;
+    if (!ensure(next_v, bars.kv_full(sv), kpv) || !ensure(next_p, bars.p_full(0, 0), pj)) {
       ok = false;
-      break;
+      return false;
     }
     bool probe = false;
 #pragma unroll
@@ -205,12 +210,12 @@ __device__ void run_mma(const AttnFp8Params& p, uint32_t smem, Bars bars, volati
       const int k0 = part * kStepsPerPart, k1 = k0 + kStepsPerPart;
       pv_steps(0, sv, k0, k1 - 1, acc);
       probe = part + 1 < kPParts ? mbar_test(bars.p_full(0, part + 1), pj)
-                                 : (more ? mbar_test(kv_bar(ik), kv_par(ik)) : true);
+                                 : (more ? mbar_test(bars.kv_full(sk), kpk) : true);
       pv_steps(0, sv, k1 - 1, k1, acc);
     }
-    if (!ok) break;
+    if (!ok) return false;
     if (more) {
-      if (!ensure(probe, kv_bar(ik), kv_par(ik))) { ok = false; break; }
+      if (!ensure(probe, bars.kv_full(sk), kpk)) { ok = false; return false; }
       qk_steps(0, sk, 0, kSteps - 1);
       probe = mbar_test(bars.p_full(1, 0), pj);
       qk_steps(0, sk, kSteps - 1, kSteps);
@@ -226,16 +231,33 @@ __device__ void run_mma(const AttnFp8Params& p, uint32_t smem, Bars bars, volati
       probe = part + 1 < kPParts ? mbar_test(bars.p_full(1, part + 1), pj) : false;
       pv_steps(1, sv, k1 - 1, k1, acc);
     }
-    if (!ok) break;
+    if (!ok) return false;
     mma_commit(bars.kv_empty(sv));
     if (more) {
       qk_steps(1, sk, 0, kSteps - 1);
-      next_v = mbar_test(kv_bar(iv + 2), kv_par(iv + 2));
+      next_v = mbar_test(bars.kv_full((sv + 2) % kStages), kpn);
       next_p = mbar_test(bars.p_full(0, 0), pj ^ 1u);
       qk_steps(1, sk, kSteps - 1, kSteps);
       mma_commit(bars.s_full(1));
       mma_commit(bars.kv_empty(sk));
     }
+    return true;
+  };
+  // Key tiles in eights: K_j and V_j take ring slots 2j % 8 and (2j+1) % 8,
+  // and a slot's phase parity repeats every eight key tiles, so within a
+  // group every slot, descriptor offset and parity is a compile-time
+  // constant of the issuing thread's instruction stream.
+  static_assert(kStages == 8, "slot pattern");
+#pragma unroll 1
+  for (int j = 0; j < p.n_kv && ok; j += 8) {
+    ok = step(j, std::integral_constant<int, 0>{});
+    if (ok && j + 1 < p.n_kv) ok = step(j + 1, std::integral_constant<int, 1>{});
+    if (ok && j + 2 < p.n_kv) ok = step(j + 2, std::integral_constant<int, 2>{});
+    if (ok && j + 3 < p.n_kv) ok = step(j + 3, std::integral_constant<int, 3>{});
+    if (ok && j + 4 < p.n_kv) ok = step(j + 4, std::integral_constant<int, 4>{});
+    if (ok && j + 5 < p.n_kv) ok = step(j + 5, std::integral_constant<int, 5>{});
+    if (ok && j + 6 < p.n_kv) ok = step(j + 6, std::integral_constant<int, 6>{});
+    if (ok && j + 7 < p.n_kv) ok = step(j + 7, std::integral_constant<int, 7>{});
   }
   if (ok) {
     mma_commit(bars.o_full(0));
@@ -444,7 +466,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_holder;
+  // Read through a shuffle, so that the compiler knows the TMEM base to be
+  // warp-uniform (the tcgen05 addresses derived from it stay in uniform
+  // registers).
+  const uint32_t tmem = __shfl_sync(0xffffffffu, *tmem_holder, 0);
 
   if (warp >= 8) {
     regs_decrease<kCtlRegs>();

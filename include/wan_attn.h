@@ -78,8 +78,10 @@ typedef enum {
   WAN_ERR_KERNEL_IMAGE = 11,      /* a compiled attention kernel's register count differs from
                                      the one its per-warpgroup register split was written for
                                      (a toolkit other than the one the library targets) */
-  WAN_ERR_TOO_LARGE = 12          /* the step does not fit wan_dit_attn_host_static's device
+  WAN_ERR_TOO_LARGE = 12,         /* the step does not fit wan_dit_attn_host_static's device
                                      buffer (WAN_HOST_STATIC_MAX_ELEMENTS) */
+  WAN_ERR_BOUNDS = 13             /* a device-side index check of the debug-bounds build failed
+                                     (see wan_debug_bounds) */
 } wan_status;
 
 /* wan_dit_attn_host flag: the call does not wait for earlier work on
@@ -418,6 +420,27 @@ WAN_API int32_t wan_dit_attn_host_static(const void* qkv_host, void* out_host, i
  * NULL, WAN_ERR_LAUNCH when the stream reports a CUDA error.
  */
 WAN_API int32_t wan_device_error(void* stream, int32_t* code);
+
+/*
+ * Debug-bounds build (libwanattn_debug.so, compiled with WAN_DEBUG_BOUNDS):
+ * every instrumented global- and shared-memory access of the kernels checks
+ * its element range against the extent of its buffer as the launch
+ * parameters define it; a failed check records the site and offset, counts
+ * the failure and skips the access (no trap: the context stays usable). The
+ * pages have no counterpart: this stands in for a memory checker, which this
+ * library cannot rely on being available.
+ *
+ * Synchronises `stream`, then reads and clears the records of every kernel
+ * file. *enabled = 1 in the debug-bounds build, 0 in the release build (which
+ * records nothing and touches no device). *first_fault is 0 when no check
+ * failed, else the first failure of the first kernel file that has one: the
+ * site in bits 56-63 (debug_bounds.cuh names them) and the element offset's
+ * low 56 bits; *count is the number of failed checks. Like wan_device_error's
+ * words, the records are one set per device, shared by every launch on it.
+ * Returns WAN_ERR_BOUNDS when *count != 0, WAN_ERR_NULL when a pointer is
+ * NULL, WAN_ERR_LAUNCH when a CUDA call fails.
+ */
+WAN_API int32_t wan_debug_bounds(void* stream, int32_t* enabled, uint64_t* first_fault, uint64_t* count);
 
 /*
  * Self-test of failure detection. Launches the attention kernel exactly as

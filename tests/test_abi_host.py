@@ -39,8 +39,8 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings(lib):
-    assert lib.wan_abi_version() == 11
-    for code in range(13):
+    assert lib.wan_abi_version() == 12
+    for code in range(14):
         assert lib.wan_status_string(code)
     assert lib.wan_status_string(99) == b"unknown status"
 
@@ -241,7 +241,7 @@ C_CALLER = r"""
 int main(void) {
   int32_t s;
   printf("abi %d\n", (int)wan_abi_version());
-  for (s = 0; s <= 12; ++s) printf("status %d %s\n", (int)s, wan_status_string(s));
+  for (s = 0; s <= 13; ++s) printf("status %d %s\n", (int)s, wan_status_string(s));
   /* argument errors are reported before any CUDA call */
   printf("null %d\n", (int)wan_qk_norm_rope(NULL, 1, 1, 1, 1, 1, 128, NULL, NULL, 1e-6f, 1e4f, NULL));
   printf("head_dim %d\n", (int)wan_self_attention((const void*)16, (void*)4096, 1, 1, 1, 64, 0.f, NULL));
@@ -268,10 +268,10 @@ def test_header_compiles_as_c_and_links(lib, tmp_path):
                     "-Wl,-rpath," + libdir], check=True, capture_output=True)
     out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.splitlines()
     assert out[0] == f"abi {lib.wan_abi_version()}"
-    texts = [line.split(" ", 2)[2] for line in out[1:14]]
-    assert all(texts) and len(set(texts)) == 13
-    assert out[14] == "null 1"          # WAN_ERR_NULL
-    assert out[15] == "head_dim 4"      # WAN_ERR_HEAD_DIM
+    texts = [line.split(" ", 2)[2] for line in out[1:15]]
+    assert all(texts) and len(set(texts)) == 14
+    assert out[15] == "null 1"          # WAN_ERR_NULL
+    assert out[16] == "head_dim 4"      # WAN_ERR_HEAD_DIM
 
 
 def test_build_refuses_a_split_register_kernel_with_another_register_count():

@@ -29,10 +29,15 @@ THETA = 10000.0
 STATUS = {0: "WAN_OK", 1: "WAN_ERR_NULL", 2: "WAN_ERR_ALIGN", 3: "WAN_ERR_SHAPE",
           4: "WAN_ERR_HEAD_DIM", 5: "WAN_ERR_PARAM", 6: "WAN_ERR_UNSUPPORTED_DEVICE",
           7: "WAN_ERR_LAUNCH", 8: "WAN_ERR_DEVICE_TIMEOUT", 9: "WAN_ERR_ALIAS",
-          10: "WAN_ERR_MEMORY_KIND", 11: "WAN_ERR_KERNEL_IMAGE", 12: "WAN_ERR_TOO_LARGE"}
+          10: "WAN_ERR_MEMORY_KIND", 11: "WAN_ERR_KERNEL_IMAGE", 12: "WAN_ERR_TOO_LARGE",
+          13: "WAN_ERR_BOUNDS"}
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-_LIB_PATH = os.path.join(_HERE, "_lib", "libwanattn.so")
+# WAN_DEBUG_BOUNDS=1 in the environment selects the debug-bounds build
+# (device-side index checks; see debug_bounds()), built by
+# `python -m video_diffusion_transformer_packed_b200.build --debug-bounds`.
+_LIB_PATH = os.path.join(_HERE, "_lib", "libwanattn_debug.so" if os.environ.get("WAN_DEBUG_BOUNDS") == "1"
+                         else "libwanattn.so")
 _lib = None
 _lock = threading.Lock()
 
@@ -104,6 +109,9 @@ def load_library() -> ctypes.CDLL:
             lib.wan_attention_merge.restype = I32
             lib.wan_dit_attn_host_static.argtypes = [P, P, I64, I32, I32, I32, I32, I32, P, P, F, F, F, I32, I32, P]
             lib.wan_dit_attn_host_static.restype = I32
+            lib.wan_debug_bounds.argtypes = [P, ctypes.POINTER(I32), ctypes.POINTER(ctypes.c_uint64),
+                                             ctypes.POINTER(ctypes.c_uint64)]
+            lib.wan_debug_bounds.restype = I32
             _lib = lib
     return _lib
 
@@ -506,6 +514,30 @@ def selftest_wait_timeout(qkv, heads: int, out=None, wait_limit_ns: int = 20_000
                                                     heads, HEAD_DIM, int(wait_limit_ns), _stream(stream)),
            "wan_selftest_wait_timeout")
     return out
+
+
+def debug_bounds(stream=None):
+    """Reads and clears the debug-bounds records (wan_debug_bounds): returns
+    (enabled, count, site, offset) -- enabled is False for the release build,
+    which records nothing and touches no device; site and offset name the
+    first failed check (0, 0 when none failed)."""
+    lib = load_library()
+    handle = 0
+    if stream is not None:
+        handle = _stream(stream)
+    else:
+        import torch
+        if torch.cuda.is_available():
+            handle = _stream(None)
+    en, first, count = ctypes.c_int32(0), ctypes.c_uint64(0), ctypes.c_uint64(0)
+    st = lib.wan_debug_bounds(ctypes.c_void_p(handle), ctypes.byref(en), ctypes.byref(first), ctypes.byref(count))
+    if st not in (0, 13):
+        raise WanError(st, "wan_debug_bounds")
+    rec = first.value
+    off = rec & ((1 << 56) - 1)
+    if off >= 1 << 55:
+        off -= 1 << 56
+    return bool(en.value), count.value, rec >> 56, off if rec else 0
 
 
 def device_error(stream=None) -> int:

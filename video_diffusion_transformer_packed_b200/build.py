@@ -1,6 +1,6 @@
 """Builds the in-tree C-ABI library libwanattn.so for sm_100a with nvcc.
 
-    python -m video_diffusion_transformer_packed_b200.build [--force] [--verbose]
+    python -m video_diffusion_transformer_packed_b200.build [--force] [--verbose] [--debug-bounds]
 
 The library is self-contained (static CUDA runtime, driver entry points
 resolved at run time), so it loads on a machine without a GPU.
@@ -19,8 +19,10 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 SOURCES = ["abi.cu", "qk_norm_rope.cu", "attn_fwd.cu", "host_pipeline.cu", "fp8_quant.cu", "attn_fwd_fp8.cu", "gemm_bf16.cu",
            "attn_merge.cu", "host_static.cu"]
-HEADERS = ["sm100.cuh", "wan_kernels.h"]
+HEADERS = ["sm100.cuh", "wan_kernels.h", "debug_bounds.cuh"]
 LIB = os.path.join(PKG, "_lib", "libwanattn.so")
+# The debug-bounds build: device-side index checks (debug_bounds.cuh) compiled in.
+LIB_DEBUG = os.path.join(PKG, "_lib", "libwanattn_debug.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -38,10 +40,10 @@ def _inputs():
     return files
 
 
-def stale() -> bool:
-    if not os.path.exists(LIB):
+def stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(f) > t for f in _inputs())
 
 
@@ -72,11 +74,15 @@ def check_register_splits(ptxas_log: str) -> None:
                                f"the split, or build with the toolkit the source was tuned for.")
 
 
-def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
-    if not force and not stale():
-        return LIB
-    os.makedirs(os.path.dirname(LIB), exist_ok=True)
-    tmp = LIB + f".{os.getpid()}.tmp"
+def build(force: bool = False, verbose: bool = False, extra_flags=(), debug_bounds: bool = False) -> str:
+    """Builds libwanattn.so, or with debug_bounds the checked libwanattn_debug.so."""
+    lib = LIB_DEBUG if debug_bounds else LIB
+    if debug_bounds:
+        extra_flags = (*extra_flags, "-DWAN_DEBUG_BOUNDS")
+    if not force and not stale(lib):
+        return lib
+    os.makedirs(os.path.dirname(lib), exist_ok=True)
+    tmp = lib + f".{os.getpid()}.tmp"
     cmd = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
            "-Xcompiler", "-fvisibility=hidden", "--expt-relaxed-constexpr",
            "-I", os.path.join(ROOT, "include"), "-Xptxas", "-v", *extra_flags]
@@ -91,14 +97,15 @@ def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
     except RuntimeError:
         os.remove(tmp)
         raise
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true")
+    ap.add_argument("--debug-bounds", action="store_true", help="build the checked libwanattn_debug.so")
     a = ap.parse_args()
-    print(build(force=a.force, verbose=a.verbose))
+    print(build(force=a.force, verbose=a.verbose, debug_bounds=a.debug_bounds))
     sys.exit(0)

@@ -11,7 +11,7 @@
 
 namespace {
 
-constexpr int32_t kAbiVersion = 11;
+constexpr int32_t kAbiVersion = 12;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -191,6 +191,7 @@ const char* wan_status_string(int32_t status) {
       return "a host buffer is not page-locked, or a device buffer is not memory of the current device";
     case WAN_ERR_TOO_LARGE:
       return "the step does not fit wan_dit_attn_host_static's device buffer (WAN_HOST_STATIC_MAX_ELEMENTS)";
+    case WAN_ERR_BOUNDS: return "a device-side index check of the debug-bounds build failed (wan_debug_bounds)";
     case WAN_ERR_KERNEL_IMAGE:
       return "a compiled attention kernel's register count differs from the one its register split was "
              "written for: rebuild the library with the CUDA toolkit it targets";
@@ -626,6 +627,34 @@ int32_t wan_selftest_wait_timeout(const void* qkv, void* out, int64_t batch, int
     return WAN_ERR_LAUNCH;
   }
   return WAN_OK;
+}
+
+int32_t wan_debug_bounds(void* stream, int32_t* enabled, uint64_t* first_fault, uint64_t* count) {
+  if (!enabled || !first_fault || !count) return WAN_ERR_NULL;
+  *first_fault = 0;
+  *count = 0;
+#ifdef WAN_DEBUG_BOUNDS
+  *enabled = 1;
+  using Words = cudaError_t (*)(unsigned long long**);
+  const Words files[] = {wan::bounds_words_norm, wan::bounds_words_attn, wan::bounds_words_fp8,
+                         wan::bounds_words_quant, wan::bounds_words_gemm, wan::bounds_words_merge};
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return WAN_ERR_LAUNCH;
+  for (Words words : files) {
+    unsigned long long* w = nullptr;
+    unsigned long long h[2] = {0ull, 0ull};
+    if (words(&w) != cudaSuccess || cudaMemcpy(h, w, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess ||
+        cudaMemset(w, 0, sizeof(h)) != cudaSuccess) {
+      return WAN_ERR_LAUNCH;
+    }
+    if (*first_fault == 0) *first_fault = h[0];
+    *count += h[1];
+  }
+  return *count != 0 ? WAN_ERR_BOUNDS : WAN_OK;
+#else
+  (void)stream;
+  *enabled = 0;
+  return WAN_OK;
+#endif
 }
 
 int32_t wan_device_error(void* stream, int32_t* code) {

@@ -40,8 +40,11 @@
 #include <mutex>
 #include <type_traits>
 
+#include "debug_bounds.cuh"
 #include "sm100.cuh"
 #include "wan_kernels.h"
+
+WAN_BOUNDS_WORDS(bounds_words_attn)
 
 namespace wan {
 namespace {
@@ -116,6 +119,7 @@ struct AttnParams {
   float scale_log2; // scale * log2(e)
   uint64_t wait_ns; // limit of each pipeline wait
   int32_t skip_loads;  // self-test: the producer starts no copies, so the waits run out
+  int64_t out_units;   // (row, head) units out (or o_part, ml_part) holds: the debug-bounds extent
 };
 
 // Barrier addresses (32-bit shared-memory addresses, 8 bytes apart).
@@ -497,7 +501,9 @@ __device__ void run_softmax(const AttnParams& p, Bars bars, volatile int* abort,
     float4* dst = reinterpret_cast<float4*>(p.o_part + unit * kHD);
     float w_new = 1.f, w_old = 0.f;
     float2 ml = make_float2(m_run, l_run);
-    if (p.accumulate && row < p.q_rows) {
+    const bool in_o = row < p.q_rows && WAN_BOUNDS(kAttnPartO, unit * kHD, kHD, p.out_units * kHD);
+    const bool in_ml = row < p.q_rows && WAN_BOUNDS(kAttnPartML, unit, 1, p.out_units);
+    if (p.accumulate && in_ml) {
       const float2 acc = reinterpret_cast<const float2*>(p.ml_part)[unit];
       const float m = fmaxf(acc.x, m_run);
       w_old = exp2f(acc.x - m);
@@ -509,7 +515,7 @@ __device__ void run_softmax(const AttnParams& p, Bars bars, volatile int* abort,
       uint32_t o[32];
       tmem_ld32(tO + 32 * c, o);
       tmem_wait_ld();
-      if (row < p.q_rows) {
+      if (in_o) {
 #pragma unroll
         for (int v = 0; v < 8; ++v) {
           float4 r = make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
@@ -523,7 +529,7 @@ __device__ void run_softmax(const AttnParams& p, Bars bars, volatile int* abort,
         }
       }
     }
-    if (row < p.q_rows) reinterpret_cast<float2*>(p.ml_part)[unit] = ml;
+    if (in_ml) reinterpret_cast<float2*>(p.ml_part)[unit] = ml;
     return;
   } else {
   const float inv_l = 1.f / l_run;
@@ -533,7 +539,7 @@ __device__ void run_softmax(const AttnParams& p, Bars bars, volatile int* abort,
     uint32_t o[32];
     tmem_ld32(tO + 32 * c, o);
     tmem_wait_ld();
-    if (row < p.q_rows) {
+    if (row < p.q_rows && WAN_BOUNDS(kAttnOut, unit * kHD + 32 * c, 32, p.out_units * kHD)) {
       uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
 #pragma unroll
       for (int v = 0; v < 4; ++v) {
@@ -750,6 +756,7 @@ cudaError_t launch_attn_fwd(const AttnPlan& plan, cudaStream_t stream, bool pdl,
   p.nh = plan.nh;
   p.q_row0 = plan.q_row0;
   p.q_rows = plan.q_rows;
+  p.out_units = static_cast<int64_t>(plan.b0 + plan.nb) * plan.q_rows * plan.heads;
   p.q_pairs = (plan.q_rows + 2 * kBM - 1) / (2 * kBM);
   p.scale_log2 = plan.scale_log2;
   p.skip_log2 = plan.skip_threshold > 0.f ? log2f(plan.skip_threshold) : -INFINITY;

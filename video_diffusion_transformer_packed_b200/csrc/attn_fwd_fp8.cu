@@ -35,8 +35,11 @@
 #include <mutex>
 #include <type_traits>
 
+#include "debug_bounds.cuh"
 #include "sm100.cuh"
 #include "wan_kernels.h"
+
+WAN_BOUNDS_WORDS(bounds_words_fp8)
 
 namespace wan {
 namespace {
@@ -79,6 +82,7 @@ struct AttnFp8Params {
   float scale_log2;  // scale * sq * sk * log2(e)
   float out_scale;   // sv
   uint64_t wait_ns;
+  int64_t out_elems;  // elements of out: the debug-bounds extent
 };
 
 struct Bars {
@@ -408,7 +412,8 @@ __device__ void run_softmax(const AttnFp8Params& p, Bars bars, volatile int* abo
     uint32_t o[32];
     tmem_ld32(tO + 32 * c, o);
     tmem_wait_ld();
-    if (row < p.S) {
+    if (row < p.S &&
+        WAN_BOUNDS(kFp8Out, (static_cast<int64_t>(b) * p.S + row) * p.D + h * kHD + 32 * c, 32, p.out_elems)) {
       uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
 #pragma unroll
       for (int v = 0; v < 4; ++v) {
@@ -558,6 +563,7 @@ cudaError_t launch_attn_fp8(const void* qk8, const void* v8t, void* out, int64_t
   p.scale_log2 = sc * scale_q * scale_k * 1.4426950408889634f;
   p.out_scale = scale_v;
   p.wait_ns = kWaitLimitNs;
+  p.out_elems = batch * S * static_cast<int64_t>(D);
   const int64_t grid = batch * heads * static_cast<int64_t>(p.q_pairs);
   if (grid > INT32_MAX) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};

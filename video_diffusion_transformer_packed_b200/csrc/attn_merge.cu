@@ -18,7 +18,10 @@
 
 #include <cstdint>
 
+#include "debug_bounds.cuh"
 #include "wan_kernels.h"
+
+WAN_BOUNDS_WORDS(bounds_words_merge)
 
 namespace wan {
 namespace {
@@ -38,10 +41,14 @@ __global__ void __launch_bounds__(kMergeThreads)
   const int64_t unit = static_cast<int64_t>(blockIdx.x) * (kMergeThreads / 32) + (threadIdx.x >> 5);
   if (unit >= n_units) return;
   const int lane = threadIdx.x & 31;
+  if (!WAN_BOUNDS(kMergeAcc, unit * kHD + 4 * lane, 4, n_units * kHD) || !WAN_BOUNDS(kMergeAcc, 2 * unit, 2, 2 * n_units)) {
+    return;
+  }
   float4* oa = reinterpret_cast<float4*>(o_acc + unit * kHD) + lane;
   float2 mla = reinterpret_cast<const float2*>(ml_acc)[unit];
   float4 o = *oa;
-  if (o_part != nullptr) {
+  if (o_part != nullptr && WAN_BOUNDS(kMergePart, unit * kHD + 4 * lane, 4, n_units * kHD) &&
+      WAN_BOUNDS(kMergePart, 2 * unit, 2, 2 * n_units)) {
     const float2 mlp = reinterpret_cast<const float2*>(ml_part)[unit];
     const float4 op = reinterpret_cast<const float4*>(o_part + unit * kHD)[lane];
     const float m = fmaxf(mla.x, mlp.x);
@@ -51,7 +58,7 @@ __global__ void __launch_bounds__(kMergeThreads)
     *oa = o;
     if (lane == 0) reinterpret_cast<float2*>(ml_acc)[unit] = mla;
   }
-  if (out != nullptr) {
+  if (out != nullptr && WAN_BOUNDS(kMergeOut, unit * kHD + 4 * lane, 4, n_units * kHD)) {
     const float inv_l = 1.f / mla.y;
     reinterpret_cast<uint2*>(out + unit * kHD)[lane] =
         make_uint2(pack_bf16x2_rn(o.x * inv_l, o.y * inv_l), pack_bf16x2_rn(o.z * inv_l, o.w * inv_l));

@@ -16,8 +16,11 @@
 
 #include <cstdint>
 
+#include "debug_bounds.cuh"
 #include "sm100.cuh"
 #include "wan_kernels.h"
+
+WAN_BOUNDS_WORDS(bounds_words_quant)
 
 namespace wan {
 namespace {
@@ -51,9 +54,12 @@ __global__ void __launch_bounds__(kThreads)
     const int t = idx >> 4, c = idx & 15;  // token in the tile, 8-element chunk of the head
     const int s = s0 + t;
     uint4 v = make_uint4(0, 0, 0, 0);
-    if (s < S) {
-      const uint16_t* src = qkv + (static_cast<int64_t>(b) * S + s) * 3 * D + h * 128 + c * 8;
-      uint8_t* dst = qk8 + (static_cast<int64_t>(b) * S + s) * 2 * D + h * 128 + c * 8;
+    const int64_t src_off = (static_cast<int64_t>(b) * S + s) * 3 * D + h * 128 + c * 8;
+    const int64_t dst_off = (static_cast<int64_t>(b) * S + s) * 2 * D + h * 128 + c * 8;
+    if (s < S && WAN_BOUNDS(kQuantLoad, src_off, 2 * D + 8, static_cast<int64_t>(gridDim.z) * S * 3 * D) &&
+        WAN_BOUNDS(kQuantStoreQK, dst_off, D + 8, static_cast<int64_t>(gridDim.z) * S * 2 * D)) {
+      const uint16_t* src = qkv + src_off;
+      uint8_t* dst = qk8 + dst_off;
       const uint4 q = *reinterpret_cast<const uint4*>(src);
       const uint4 k = *reinterpret_cast<const uint4*>(src + D);
       v = *reinterpret_cast<const uint4*>(src + 2 * D);
@@ -64,7 +70,9 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       const uint32_t w = e < 4 ? cv.x : cv.y;
-      vt[(c * 8 + e) * kVtPitch + t] = static_cast<uint8_t>(w >> (8 * (e & 3)));
+      if (WAN_BOUNDS(kQuantStageV, (c * 8 + e) * kVtPitch + t, 1, 128 * kVtPitch)) {
+        vt[(c * 8 + e) * kVtPitch + t] = static_cast<uint8_t>(w >> (8 * (e & 3)));
+      }
     }
   }
   __syncthreads();
@@ -75,6 +83,10 @@ __global__ void __launch_bounds__(kThreads)
     const int d = idx >> 3, c = idx & 7;
     const int64_t col = s0 + c * 16;
     if (col >= s_pitch) continue;
+    if (!WAN_BOUNDS(kQuantStoreV, ((static_cast<int64_t>(b) * heads + h) * 128 + d) * s_pitch + col, 16,
+                    static_cast<int64_t>(gridDim.z) * heads * 128 * s_pitch)) {
+      continue;
+    }
     *reinterpret_cast<uint4*>(vrow + d * s_pitch + col) =
         *reinterpret_cast<const uint4*>(&vt[d * kVtPitch + c * 16]);
   }
@@ -89,6 +101,9 @@ __global__ void __launch_bounds__(kThreads)
   for (int64_t tok = blockIdx.x; tok < tokens; tok += gridDim.x) {
     const uint4* row = reinterpret_cast<const uint4*>(qkv + tok * 3 * static_cast<int64_t>(D));
     for (int c = threadIdx.x; c < chunks; c += kThreads) {
+      if (!WAN_BOUNDS(kAmaxLoad, tok * 3 * static_cast<int64_t>(D) + 8 * c, 8, tokens * 3 * static_cast<int64_t>(D))) {
+        continue;
+      }
       const uint4 v = row[c];
       const int which = (c * 8) / D;
       float a = fmaxf(fmaxf(fabsf(bf_lo(v.x)), fabsf(bf_hi(v.x))), fmaxf(fabsf(bf_lo(v.y)), fabsf(bf_hi(v.y))));

@@ -37,8 +37,11 @@
 #include <cstring>
 #include <mutex>
 
+#include "debug_bounds.cuh"
 #include "sm100.cuh"
 #include "wan_kernels.h"
+
+WAN_BOUNDS_WORDS(bounds_words_gemm)
 
 namespace wan {
 namespace {
@@ -258,13 +261,17 @@ __global__ void __launch_bounds__(kThreads, 1)
               ss += __hiloint2double(static_cast<int>(__umulhi(__float_as_uint(hi * hi), 1u << 29) + 0x38000000u), 0);
             }
           }
-          if (row < p.M) {
+          if (row < p.M && WAN_BOUNDS(kGemmY, row * p.N + static_cast<int64_t>(nb) * kTileN + 32 * c, 32,
+                                      static_cast<int64_t>(p.M) * p.N)) {
             uint4* dst = reinterpret_cast<uint4*>(yrow + 32 * c);
 #pragma unroll
             for (int q = 0; q < 4; ++q) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
           }
         }
-        if (stat && row < p.M) p.stats[row * p.stat_tiles + nb] = ss;
+        if (stat && row < p.M &&
+            WAN_BOUNDS(kGemmStats, row * p.stat_tiles + nb, 1, static_cast<int64_t>(p.M) * p.stat_tiles)) {
+          p.stats[row * p.stat_tiles + nb] = ss;
+        }
       }
       tc_fence_before();
       mbar_arrive(bars.acc_empty());

@@ -45,8 +45,11 @@
 #include <cstdint>
 #include <mutex>
 
+#include "debug_bounds.cuh"
 #include "sm100.cuh"
 #include "wan_kernels.h"
+
+WAN_BOUNDS_WORDS(bounds_words_norm)
 
 namespace wan {
 namespace {
@@ -305,7 +308,8 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const __grid_
   if (tid == 0) {
     for (int s = 0; s < p.stages; ++s) {
       const int64_t tok = t_begin + s;
-      if (tok < t_end) {
+      if (tok < t_end &&
+          WAN_BOUNDS(kNormLoad, tok * 3 * static_cast<int64_t>(p.D), 2 * p.D, p.tokens * 3 * static_cast<int64_t>(p.D))) {
         const uint32_t bar = smem_u32(&tail.full[s]);
         mbar_arrive_expect_tx(bar, p.stage_bytes);
         bulk_load(ring + s * p.stage_bytes, p.qkv + tok * 3 * static_cast<int64_t>(p.D), p.stage_bytes, bar);
@@ -350,7 +354,10 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const __grid_
     // partial sum now; the load's latency hides behind the ring wait.
     double st_part = 0.0;
     if constexpr (kStats) {
-      if (lane < p.stat_half) st_part = p.stats[tok * p.stat_row + which * p.stat_half + lane];
+      if (lane < p.stat_half &&
+          WAN_BOUNDS(kNormStats, tok * p.stat_row + which * p.stat_half + lane, 1, p.tokens * p.stat_row)) {
+        st_part = p.stats[tok * p.stat_row + which * p.stat_half + lane];
+      }
     }
     // The next token's rotations, ahead of time (they do not depend on the data).
     const int rnext = rbuf == 2 ? 0 : rbuf + 1;
@@ -378,7 +385,9 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const __grid_
 #pragma unroll
     for (int k = 0; k < VPT; ++k) {
       const int vi = u + kRowThreads * k;
-      v[k] = vi < p.nvec ? ld_shared_v4(src + 16 * vi) : make_uint4(0, 0, 0, 0);
+      v[k] = vi < p.nvec && WAN_BOUNDS(kNormStage, which * p.D * 2 + 16 * vi, 16, static_cast<int64_t>(p.stage_bytes))
+                 ? ld_shared_v4(src + 16 * vi)
+                 : make_uint4(0, 0, 0, 0);
     }
 
     if constexpr (!kStats) {
@@ -400,7 +409,8 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const __grid_
 
     if (tid == 0) {
       const int64_t next = tok + p.stages;
-      if (next < t_end) {
+      if (next < t_end &&
+          WAN_BOUNDS(kNormLoad, next * 3 * static_cast<int64_t>(p.D), 2 * p.D, p.tokens * 3 * static_cast<int64_t>(p.D))) {
         const uint32_t bar = smem_u32(&tail.full[stage]);
         mbar_arrive_expect_tx(bar, p.stage_bytes);
         bulk_load(ring + stage * p.stage_bytes, p.qkv + next * 3 * static_cast<int64_t>(p.D),
@@ -433,7 +443,7 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const __grid_
     for (int k = 0; k < VPT; ++k) {
       const int vi = u + kRowThreads * k;
       // gammas: L1-resident, the same channels for every token
-      const uint4 gv = vi < p.nvec ? ld_cached(g + 8 * vi) : make_uint4(0, 0, 0, 0);
+      const uint4 gv = vi < p.nvec && WAN_BOUNDS(kNormGamma, 8 * vi, 8, p.D) ? ld_cached(g + 8 * vi) : make_uint4(0, 0, 0, 0);
       const uint32_t xw[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
       const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
       uint32_t near = 0xFFFFFFFFu;
@@ -464,7 +474,9 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const __grid_
 #pragma unroll
     for (int k = 0; k < VPT; ++k) {
       const int vi = u + kRowThreads * k;
-      if (vi < p.nvec) st_v4(x + 8 * vi, make_uint4(y[k][0], y[k][1], y[k][2], y[k][3]));
+      if (vi < p.nvec && WAN_BOUNDS(kNormStore, tok, 1, p.tokens) && WAN_BOUNDS(kNormColumn, 8 * vi, 8, p.D)) {
+        st_v4(x + 8 * vi, make_uint4(y[k][0], y[k][1], y[k][2], y[k][3]));
+      }
     }
     rbuf = rnext;
     if (++stage == p.stages) {

@@ -154,4 +154,13 @@ cudaError_t norm_error_word(int** word);
 cudaError_t fp8_error_word(int** word);
 cudaError_t gemm_error_word(int** word);
 
+// Debug-bounds records of each kernel file (debug_bounds.cuh): two words,
+// the first failed check and the count of failures.
+cudaError_t bounds_words_norm(unsigned long long** words);
+cudaError_t bounds_words_attn(unsigned long long** words);
+cudaError_t bounds_words_fp8(unsigned long long** words);
+cudaError_t bounds_words_quant(unsigned long long** words);
+cudaError_t bounds_words_gemm(unsigned long long** words);
+cudaError_t bounds_words_merge(unsigned long long** words);
+
 }  // namespace wan

@@ -1,4 +1,4 @@
-"""The FP8 attention kernel evaluates 2^x for a quarter of its probabilities
+"""The FP8 attention kernel evaluates 2^x for an eighth of its probabilities
 with a polynomial on the FMA pipe. Checks, on the CPU: the embedded coefficients are
 the ones exp2_poly.py fits; the fit is minimax (equioscillating) with max
 relative error below 1e-4; and the kernel's float32 steps (magic-number

@@ -7,7 +7,7 @@ oracle, which works on the dequantised codes; what differs is that the kernel
 rounds each probability p_j (normalised so that the row's largest is at least
 1) to e4m3 before the P V product: |p^_j - p_j| <= max(2^-4 p_j, 2^-10)
 (relative in e4m3's normal range, absolute in its subnormal range), plus the
-relative error of the exponential itself (below 1.2e-4 for the quarter the
+relative error of the exponential itself (below 1.2e-4 for the eighth the
 kernel evaluates with its polynomial, far smaller for MUFU ex2). With the
 row sum taken over the unrounded p_j, every output element then obeys
   |o^_i - o_i| <= sum_j max((2^-4 + 1.2e-4) p_j, 2^-10) |v_j| / sum_j p_j

@@ -273,9 +273,9 @@ __device__ void run_mma(const AttnFp8Params& p, uint32_t smem, Bars bars, volati
   if (!mbar_wait(bars.drain(), 0, nullptr, kWaitLimitNs)) atomicOr(&g_attn_fp8_error_word, kErrDrain);
 }
 
-// 2^x on the FMA pipe for a quarter of the exponentials (MUFU ex2 gives 16
+// 2^x on the FMA pipe for an eighth of the exponentials (MUFU ex2 gives 16
 // per clock per SM, as many cycles per tile as the fp8 products need twice
-// over): x = n + f, n = round(x) by the 1.5*2^23 magic add, f in [-1/2, 1/2];
+// over; a larger share costs more FMA/ALU issue than it saves): x = n + f, n = round(x) by the 1.5*2^23 magic add, f in [-1/2, 1/2];
 // 2^x = 2^n * p(f) with p the degree-3 minimax fit of 2^f in relative error
 // (7.5e-5) that exp2_poly.py next to this file computes; 2^n is applied by
 // adding n to the exponent field. x is clamped at -126 (masked keys).
@@ -300,8 +300,8 @@ __device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
   const float r1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(j1) << 23));
   return f2(r0, r1);
 }
-// Four-key groups whose exponentials take the polynomial: one in four.
-__host__ __device__ constexpr bool poly_group(int w) { return (w & 3) == 3; }
+// Four-key groups whose exponentials take the polynomial: one in eight.
+__host__ __device__ constexpr bool poly_group(int w) { return (w & 7) == 7; }
 
 // ----------------------------------------------------------------- softmax
 __device__ void run_softmax(const AttnFp8Params& p, Bars bars, volatile int* abort, uint32_t tmem, int t,

@@ -342,6 +342,11 @@ WAN_API int32_t wan_dit_attn(void* qkv, void* out, int64_t batch, int32_t F, int
  * in and out and the kernels on three internal streams per device. Calls on
  * one device are serialised while they are enqueued, and their kernels run in
  * that order.
+ * Ownership: all four buffers stay the caller's. They must stay allocated, and
+ * qkv_host unmodified, until `stream` has passed this call: the copies read
+ * qkv_host and write out_host after the call returns. A pinned-memory cache
+ * that recycles a freed block at once (as PyTorch's does for memory it did not
+ * see in use) must not get qkv_host back before then.
  * Errors: argument errors return before anything is enqueued, as for the other
  * calls; WAN_ERR_MEMORY_KIND when a host buffer is not page-locked or a device
  * buffer is not memory of the current device; WAN_ERR_LAUNCH when the runtime

@@ -162,3 +162,24 @@ def test_overlapped_calls_when_kernels_outlast_the_transfer(n_sets):
     assert wan.device_error() == 0
     for o, r in zip(outs, refs):
         assert torch.equal(o.view(torch.int16), r.view(torch.int16))
+
+
+def test_temporary_pinned_input_survives_until_the_step_is_done():
+    """The input's copies run on the library's streams after the call returns.
+    A temporary pinned input must not go back to torch's pinned-memory cache
+    (which would hand the same block to the next pin_memory() at once) before
+    they are done: the returned output keeps it referenced. Same-size pinned
+    buffers filled with other data right after the call would take its block
+    otherwise; the result must still be the step of the original input."""
+    w = wi.Workload("case", 2, (5, 20, 26), 8)
+    qkv, gq, gk = wi.inputs_for(w, seed=71)
+    gq_d, gk_d = gq.cuda(), gk.cuda()
+    ref = wan.dit_attn(qkv.cuda(), w.grid, w.heads, gq_d, gk_d).cpu()
+    s = torch.cuda.Stream()
+    for trial in range(5):  # without the reference, 2 of 5 such trials read recycled data
+        with torch.cuda.stream(s):
+            out_h = wan.dit_attn_host(qkv.contiguous().pin_memory(), w.grid, w.heads, gq_d, gk_d, stream=s)
+            others = [torch.full_like(qkv, float(k + 3)).pin_memory() for k in range(4)]
+        s.synchronize()
+        assert torch.equal(out_h.view(torch.int16), ref.view(torch.int16)), trial
+        assert all(float(o[0, 0, 0]) == k + 3 for k, o in enumerate(others))

@@ -442,8 +442,9 @@ def dit_attn_host(qkv_host, grid: Sequence[int], heads: int, gamma_q, gamma_k, o
     qk_norm_rope, self_attention and the device->host copy of the output,
     overlapped chunk by chunk inside the library. qkv_dev / out_dev are the
     device buffers it runs through (allocated on the current device when not
-    given); qkv_host is only read. Asynchronous on `stream`: synchronise it
-    before reading out_host. overlap_input: the call does not wait for earlier
+    given); qkv_host is only read, asynchronously (the returned out_host keeps a
+    reference to it until it is freed). Asynchronous on `stream`: synchronise
+    it before reading out_host. overlap_input: the call does not wait for earlier
     work on `stream`; it still waits for earlier calls of this function that
     use the same device buffers (the caller guarantees nothing else does), so
     alternating two buffer sets overlaps one call's input transfer with the
@@ -473,6 +474,11 @@ def dit_attn_host(qkv_host, grid: Sequence[int], heads: int, gamma_q, gamma_k, o
                                             _bf16_cuda(gamma_k, "gamma_k"), eps, theta, scale,
                                             int(heads_per_chunk), 1 if overlap_input else 0, _stream(stream)),
            "wan_dit_attn_host")
+    # The copies out of qkv_host run on the library's own streams, which
+    # torch's pinned-memory cache does not see: a temporary qkv_host freed
+    # now could be handed to another pin_memory() and overwritten while it
+    # is still being read. The output keeps it alive.
+    out_host._wan_source = qkv_host
     return out_host
 
 
@@ -498,6 +504,7 @@ def dit_attn_host_static(qkv_host, grid: Sequence[int], heads: int, gamma_q, gam
                                                    _bf16_cuda(gamma_k, "gamma_k"), eps, theta, scale,
                                                    int(heads_per_chunk), 1 if overlap_input else 0,
                                                    _stream(stream)), "wan_dit_attn_host_static")
+    out_host._wan_source = qkv_host  # read asynchronously: see dit_attn_host
     return out_host
 
 

@@ -183,3 +183,30 @@ def test_temporary_pinned_input_survives_until_the_step_is_done():
         s.synchronize()
         assert torch.equal(out_h.view(torch.int16), ref.view(torch.int16)), trial
         assert all(float(o[0, 0, 0]) == k + 3 for k, o in enumerate(others))
+
+
+def test_device_temporaries_stay_reserved_while_a_side_stream_step_runs():
+    """Called on a stream other than torch's current one and without device
+    buffers, the step makes qkv_dev and out_dev itself and drops them when
+    the call returns, while its copies and kernels still run. Tensors of the
+    same sizes allocated on the current stream right after the call, and
+    overwritten there while the step runs, must not get their memory: the
+    result must still be the step of the input."""
+    w = wi.Workload("case", 1, (21, 30, 52), 2)  # S = 32760: about a millisecond each of copy and attention
+    qkv, gq, gk = wi.inputs_for(w, seed=73)
+    gq_d, gk_d = gq.cuda(), gk.cuda()
+    ref = wan.dit_attn(qkv.cuda(), w.grid, w.heads, gq_d, gk_d).cpu()
+    qkv_p = _pinned(qkv)
+    s = torch.cuda.Stream()
+    torch.cuda.synchronize()
+    for trial in range(3):
+        out_h = wan.dit_attn_host(qkv_p, w.grid, w.heads, gq_d, gk_d, stream=s)
+        a = torch.empty(qkv.shape, dtype=torch.bfloat16, device="cuda")
+        o = torch.empty((w.batch, w.seq_len, w.dim), dtype=torch.bfloat16, device="cuda")
+        for k in range(6):  # overwrite both at intervals spanning the step
+            torch.cuda._sleep(400_000)
+            a.fill_(float(k + 1))
+            o.fill_(float(-k - 1))
+        s.synchronize()
+        torch.cuda.synchronize()
+        assert torch.equal(out_h.view(torch.int16), ref.view(torch.int16)), trial

@@ -128,6 +128,19 @@ def _stream(stream) -> int:
     return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
 
 
+def _on_stream(stream, device):
+    """Context that makes `stream` (a torch stream, an object with a
+    `cuda_stream` handle, a raw cudaStream_t, or None for the current stream)
+    torch's current stream on `device`."""
+    import contextlib
+    import torch
+    if stream is None:
+        return contextlib.nullcontext()
+    if not isinstance(stream, torch.cuda.Stream):
+        stream = torch.cuda.ExternalStream(_stream(stream), device=device)
+    return torch.cuda.stream(stream)
+
+
 def _check_packed(qkv, heads: int, grid=None) -> None:
     """Shapes the C ABI cannot see (it takes raw pointers): refuse mismatches
     here, before anything is launched."""
@@ -458,10 +471,15 @@ def dit_attn_host(qkv_host, grid: Sequence[int], heads: int, gamma_q, gamma_k, o
     dev = gamma_q.device
     if out_host is None:
         out_host = torch.empty((B, S, heads * HEAD_DIM), dtype=torch.bfloat16).pin_memory()
-    if qkv_dev is None:
-        qkv_dev = torch.empty(qkv_host.shape, dtype=torch.bfloat16, device=dev)
-    if out_dev is None:
-        out_dev = torch.empty((B, S, heads * HEAD_DIM), dtype=torch.bfloat16, device=dev)
+    # Device buffers made here are dropped when the call returns, while the
+    # library's streams still use them. Allocated on the call's stream, which
+    # the library makes wait for its last copy, torch's caching allocator
+    # hands their memory out again only in that stream's order.
+    with _on_stream(stream, dev):
+        if qkv_dev is None:
+            qkv_dev = torch.empty(qkv_host.shape, dtype=torch.bfloat16, device=dev)
+        if out_dev is None:
+            out_dev = torch.empty((B, S, heads * HEAD_DIM), dtype=torch.bfloat16, device=dev)
     _check_out(out_host, qkv_host, heads)
     _check_packed(qkv_dev, heads, grid)
     if tuple(qkv_dev.shape) != tuple(qkv_host.shape):

@@ -59,3 +59,32 @@ def test_reference_arm_runs_on_rank0_only(monkeypatch, capsys):
     args = type("A", (), {"workload": "tiny_5x8x8_h12_b1", "steps": 1, "warmup": 0, "gpus": 2})()
     assert bench.run_reference(args) == 0
     assert capsys.readouterr().out == ""
+
+
+def test_reference_arm_line_carries_the_contract_keys(monkeypatch, capsys):
+    """Rank 0 prints one JSON line with the keys of the bench contract: the
+    reference tag, the metric and its unit, the run's shape, a CPU-baseline
+    object describing this run and an end-to-end object with no copies. The
+    oracle's timing itself is stubbed (it runs for seconds by design)."""
+    import json
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setattr(bench, "oracle_sample", lambda w, qkv, gq, gk, target_s: (0.02, 0.5, "stub sample"))
+    args = type("A", (), {"workload": "tiny_5x8x8_h12_b1", "steps": 3, "warmup": 1, "gpus": 1})()
+    assert bench.run_reference(args) == 0
+    out = capsys.readouterr().out.strip().splitlines()
+    assert len(out) == 1
+    line = json.loads(out[0])
+    assert line["impl"] == "reference"
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["value"] == pytest.approx(0.02) and line["unit"] == "TFLOP/s"
+    assert line["steps"] == 3 and line["warmup"] == 1 and line["n_gpus"] == 1
+    assert line["ms_per_step"] == pytest.approx(500.0)
+    assert line["higher_is_better"] is True and line["vs_baseline"] is None
+    assert line["config"]["workload"] == "tiny_5x8x8_h12_b1"
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] >= 1 and cb["sample"]
+    e2e = line["e2e"]
+    assert e2e["value"] == line["value"] and e2e["unit"] == line["unit"]
+    assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0

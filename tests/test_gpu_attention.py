@@ -171,3 +171,21 @@ def test_full_length_rising_max_sampled_rows():
     idx = wi.sample_rows(S, 4096, seed=44).numpy()
     ref = oracle.attention_rows(qkv, heads, _rows_of_head(S, idx), SCALE)
     assert_attention_close(got.view(S, HD)[torch.from_numpy(idx)], ref, "rising max, sampled rows")
+
+
+def test_full_length_equal_scores_give_the_mean_of_v():
+    """Q = 0: every score is 0 and every probability exactly 1, so each row's
+    output is the mean of V over all 32760 keys, the ragged last tile
+    included: the row sum counts 32760 ones and O sums 32760 rows of V in
+    fp32. Sampled rows against the oracle at the flat bound, and every element
+    against the closed form within the output's bf16 rounding."""
+    S, heads = LONG_S, 1
+    qkv = wi.packed_qkv(1, S, heads, seed=45)
+    qkv[0, :, :HD] = 0
+    got = gpu_attention(qkv, heads).view(S, HD).double()
+    idx = wi.sample_rows(S, 256, seed=46).numpy()
+    ref = oracle.attention_rows(qkv, heads, _rows_of_head(S, idx), SCALE)
+    assert_attention_close(got[torch.from_numpy(idx)].float(), ref, "equal scores, sampled rows")
+    mean = qkv[0, :, 2 * HD:3 * HD].double().mean(0)
+    err = (got - mean).abs()
+    assert bool((err <= 2.0 ** -8 * mean.abs() + 1e-7).all()), float(err.max())

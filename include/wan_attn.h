@@ -112,11 +112,15 @@ WAN_API int32_t wan_abi_version(void);
 /*
  * (1) Q/K RMSNorm + bf16 round + 3D RoPE, IN PLACE on the packed buffer.
  *   For every token and X in {Q, K}:
- *     r = 1/sqrt(mean_{c<D} X_c^2 + eps)      (fp32 accumulation)
- *     y_c = bf16_rne(X_c * r * gamma_X[c])
- *     pairs of y rotated by the token's (frame,row,column) angles in fp32,
- *     then rounded to bf16 and written back over X.
+ *     r = 1/sqrt(mean_{c<D} X_c^2 + eps)      (exact squares summed in fp64)
+ *     y_c = bf16_rne(X_c * r * gamma_X[c])     (correctly rounded)
+ *     pairs of y rotated by the token's (frame,row,column) angles, then
+ *     rounded to bf16 and written back over X: every element within 1 bf16
+ *     ulp of the exact definition.
  *   V is neither read nor written.
+ *   Domain: finite inputs with |X_c| < 2^64 and |X_c * gamma_X[c]| < 2^128.
+ *   The squares and the gamma products are formed exactly in fp32; larger
+ *   magnitudes overflow there and give wrong rows, with no error reported.
  * qkv      device pointer, bf16 [batch][F*H*W][3*heads*128], 16-byte aligned.
  * gamma_q, gamma_k  device pointers, bf16 [heads*128], 16-byte aligned.
  * batch >= 1; F, H, W >= 1 with F*H*W < 2^31; 1 <= heads <= WAN_MAX_HEADS;

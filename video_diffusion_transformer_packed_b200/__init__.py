@@ -170,7 +170,10 @@ def _bf16_cuda(t, name: str) -> int:
 
 def qk_norm_rope(qkv, grid: Sequence[int], heads: int, gamma_q, gamma_k, eps: float = EPS,
                  theta: float = THETA, stream=None):
-    """Q/K RMSNorm + bf16 round + 3D RoPE in place on packed qkv [B, F*H*W, 3*heads*128]."""
+    """Q/K RMSNorm + bf16 round + 3D RoPE in place on packed qkv [B, F*H*W, 3*heads*128].
+    Within 1 bf16 ulp of the exact definition for finite inputs with |x| < 2^64
+    and |x * gamma| < 2^128 (the kernel forms squares and gamma products exactly
+    in fp32; larger magnitudes overflow there)."""
     F, H, W = grid
     B = qkv.shape[0]
     _check_packed(qkv, heads, grid)

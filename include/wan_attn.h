@@ -136,6 +136,9 @@ WAN_API int32_t wan_qk_norm_rope(void* qkv, int64_t batch, int32_t F, int32_t H,
  *     out[b, i, h, :] = sum_j softmax_j(scale * q_i . k_j) v_j
  *   bf16 operands, fp32 accumulation, probabilities rounded to bf16 before
  *   the PV product, output rounded to bf16.
+ *   Domain: finite inputs whose scores scale * q_i . k_j and weighted sums stay
+ *   finite in fp32, where the tensor cores accumulate them (inputs normalised
+ *   by (1) are bounded by sqrt(heads*128) * max|gamma| per element).
  * qkv      device pointer, bf16 [batch][seq_len][3*heads*128], 16-byte aligned.
  * out      device pointer, bf16 [batch][seq_len][heads*128], 16-byte aligned,
  *          must not overlap qkv.

@@ -212,7 +212,8 @@ WAN_API int32_t wan_self_attention_fp8(const void* qk8, const void* v8t, void* o
  * projection with the distributed QK RMSNorm, "NKI kernels"): when stats is
  * not NULL, stats[row][j] = the fp64 sum of squares of the bf16 outputs of
  * row `row` in columns [256 j, 256 j + 256) (a zero output counting 2^-127,
- * as in (1)'s own sum), for j < stat_cols / 256
+ * as in (1)'s own sum; exact for outputs below 2^64 in magnitude, the domain
+ * of (1)), for j < stat_cols / 256
  * (stat_cols a multiple of 256, <= N; stats 8-byte aligned, [M][stat_cols/256]).
  */
 WAN_API int32_t wan_linear(const void* x, const void* w, void* y, int64_t M, int64_t N, int64_t K,
